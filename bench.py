@@ -1,0 +1,370 @@
+#!/usr/bin/env python
+"""Throughput of exact ring attention on B200: causal-adjusted TFLOP/s, one JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+A step is one ring_attn_fwd call over the whole workload (every query shard folds
+every KV shard in ring order). Default workload: bf16, B=1, H=8, S=1,048,576,
+D=128, P=32, causal striped. Inputs are seeded synthetic tensors resident in HBM
+(larger than L2, so no flush is needed between steps). With N>1 (torchrun) every
+rank runs its own independent instance (seed + rank): weak scaling, no collective
+on the data path; the step time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle (the correctness reference) on a
+bounded sample of query rows of the same workload; rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synthetic  # noqa: E402
+
+METRIC = "causal-adjusted attention TFLOP/s and % of B200 dense BF16 peak, 1 GPU"
+DEFAULT_WORKLOAD = "c5_bf16_s1m_striped"
+KERNEL_SRC = os.path.join(ROOT, "sequence_exact_attention_ring_b200", "csrc", "fwd_sm100.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ring_fwd_sm100_traffic.json")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synthetic.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=600))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def gather_objects(obj, world):
+    if world == 1:
+        return [obj]
+    import torch.distributed as dist
+    out = [None] * world
+    dist.all_gather_object(out, obj)
+    return out
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples of this GPU every 200 ms while the timed region runs."""
+
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
+              "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", uuid, "--query-gpu=" + ",".join(self.FIELDS), "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, flag in zip(names, parts[3:]):
+                if flag.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ peaks / traffic
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def kernel_traffic_per_launch(workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it matches the current kernel source."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as f:
+        d = json.load(f)
+    with open(KERNEL_SRC, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()
+    if d.get("kernel_source_sha256") != sha:
+        return None
+    per = d.get("bytes_per_launch", {}).get(workload)
+    return float(per) if per is not None else None
+
+
+# ------------------------------------------------------------------ CPU oracle sample
+
+def oracle_sample_rate(w, q, k, v, target_seconds: float, seed_offset: int = 0):
+    """Time the fp64 oracle on seeded query rows of one head; returns (TFLOP/s, rows, seconds, flops)."""
+    import oracle
+    from threadpoolctl import threadpool_info
+    g = torch.Generator().manual_seed(w.seed + 2000 + seed_offset)
+    b = 0
+    h = int(torch.randint(0, w.Hq, (1,), generator=g).item())
+    n_probe = 8
+    ts = sorted(torch.randperm(w.S, generator=g)[:4096].tolist())
+    picked, flops, elapsed = [], 0.0, 0.0
+    qh = q[b:b + 1, h:h + 1].cpu()
+    g_kv = h // (w.Hq // w.Hkv)
+    kh = k[b:b + 1, g_kv:g_kv + 1].cpu()
+    vh = v[b:b + 1, g_kv:g_kv + 1].cpu()
+    idx = 0
+    while idx < len(ts) and (elapsed < target_seconds):
+        batch = ts[idx: idx + n_probe]
+        idx += len(batch)
+        rows = [(0, 0, t) for t in batch]
+        t0 = time.perf_counter()
+        oracle.attention_rows(qh, kh, vh, rows, w.causal, w.scale)
+        elapsed += time.perf_counter() - t0
+        picked += batch
+        flops += sum(4.0 * w.D * ((t + 1) if w.causal else w.S) for t in batch)
+        n_probe = min(64, n_probe * 2)
+    cores = 0
+    for info in threadpool_info():
+        if info.get("user_api") == "blas":
+            cores = max(cores, int(info.get("num_threads", 0)))
+    return flops / elapsed / 1e12, len(picked), elapsed, flops, max(cores, 1), h
+
+
+# ------------------------------------------------------------------ arms
+
+def run_reference(args, world, rank):
+    """The correctness reference (fp64 CPU oracle) on bounded samples of the workload."""
+    if rank != 0:
+        return
+    w = synthetic.get(args.workload)
+    dev = "cuda" if (w.gen_device == "cuda" and torch.cuda.is_available()) else "cpu"
+    if w.gen_device == "cuda" and dev == "cpu":
+        print(json.dumps({"impl": "reference", "unavailable": "workload inputs are drawn on a CUDA device"}))
+        return
+    q, k, v = synthetic.make_inputs(w, dev)
+    per_step = max(1.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+    for i in range(args.warmup):
+        oracle_sample_rate(w, q, k, v, per_step / 4, seed_offset=i)
+    rates, rows, secs, cores = [], 0, 0.0, 1
+    for i in range(args.steps):
+        r, n, s, _, cores, _ = oracle_sample_rate(w, q, k, v, per_step, seed_offset=100 + i)
+        rates.append(r)
+        rows += n
+        secs += s
+    value = statistics.median(rates)
+    total = w.causal_flops()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total / (value * 1e12) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{rows} query rows of one head per step (fp64 oracle, full score rows), "
+                                   f"{secs:.1f} s total; ms_per_step extrapolates to the whole workload"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+
+
+def workload_config(w):
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "S": w.S, "D": w.D, "P": w.P,
+            "causal": w.causal, "layout": w.layout, "heavy_keys": w.heavy_keys,
+            "l2": "inputs larger than L2 (no flush)" if w.qkvo_bytes() > 126e6 else "L2 flushed between steps",
+            "flops_per_step": w.causal_flops()}
+
+
+def flush_l2(buf):
+    if buf is not None:
+        buf.add_(1)
+
+
+def run_ours(args, world, rank, local):
+    from sequence_exact_attention_ring_b200 import HostRunner, binding, ring_attention, status
+    w = synthetic.get(args.workload)
+    binding.load()
+    dev = torch.device("cuda", local if world > 1 else 0)
+    w_rank = synthetic.custom(w.name, w.dtype, w.B, w.Hq, w.Hkv, w.S, w.D, w.P, w.causal, w.layout,
+                              w.seed + rank, w.heavy_keys, "cuda")
+    q, k, v = synthetic.make_inputs(w_rank, dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.S), dtype=torch.float32, device=dev)
+    from sequence_exact_attention_ring_b200 import workspace_bytes
+    ws = torch.empty(workspace_bytes(q, k, w.P, w.causal, w.layout), dtype=torch.uint8, device=dev)
+    l2buf = None if w.qkvo_bytes() > 126e6 else torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        ring_attention(q, k, v, w.P, w.causal, w.layout, w.scale, out=out, lse=lse, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        flush_l2(l2buf)
+        step()
+    torch.cuda.synchronize(dev)
+    if status(ws) != 0:
+        raise RuntimeError("kernel watchdog tripped during warm-up")
+
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(dev.index)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t_start.record(stream)
+    for i in range(args.steps):
+        flush_l2(l2buf)
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    barrier(world)
+    st = status(ws)
+    elapsed_ms = t_start.elapsed_time(t_end)
+    launch_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    elapsed_ms = max_over_ranks(elapsed_ms, world)
+    launch_ms_max = max_over_ranks(launch_ms, world)
+
+    flops = w.causal_flops()
+    value = flops * world * args.steps / (elapsed_ms * 1e-3) / 1e12
+    peaks, peak_src = measured_peaks()
+    peak = float(peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"])
+    achieved = w.algorithmic_flops() / (launch_ms_max * 1e-3) / 1e12
+
+    # ---- end to end: pinned host buffers, H2D + kernel + D2H inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        qh, kh, vh = q.cpu().pin_memory(), k.cpu().pin_memory(), v.cpu().pin_memory()
+        runner = HostRunner(q.shape, k.shape, q.dtype, w.P, w.causal, w.layout, w.scale, device=dev)
+        runner.run(qh, kh, vh, stream)
+        torch.cuda.synchronize(dev)
+        del out
+        barrier(world)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e_steps = max(1, min(args.steps, 3))
+        e0.record(stream)
+        for _ in range(e_steps):
+            runner.run(qh, kh, vh, stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+        e2e = {"value": flops * world * e_steps / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": runner.h2d_bytes() * world, "d2h_bytes_per_step": runner.d2h_bytes() * world,
+               "steps": e_steps}
+
+    clocks_all = gather_objects(clocks, world)
+    statuses = gather_objects(st, world)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, n, secs, fl, cores, h = oracle_sample_rate(w, q, k, v, args.cpu_seconds)
+        cpu = {"value": rate, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+               "sample": f"{n} seeded query rows of head {h} ({fl / 1e9:.1f} GFLOP causal-adjusted, "
+                         f"{secs:.1f} s), fp64, full score rows"}
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "fp32",
+        "data": "synthetic", "config": workload_config(w),
+        "pct_of_peak": 100.0 * value / world / peak,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": kernel_traffic_per_launch(w.name),
+                     "peak_source": f"{peak_src} bf16_tflops_sustained (seconds-long kernel under the power cap)",
+                     "kernel": "ring_fwd_sm100_kernel<128>"},
+        "e2e": e2e,
+        "gpu_launches": args.steps,
+        "clocks": clocks_all[0] if world == 1 else {"per_rank": clocks_all},
+        "cpu_baseline": cpu,
+        "status": statuses,
+    }
+    print(json.dumps(line))
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,182 @@
+/*
+ * ringattn.h - C ABI of libringattn.so: exact ring attention on one B200 (sm_100a).
+ *
+ * What is computed. RingAttention (deep-architecture article on techknowgenie,
+ * section 3 "rigorous derivation of blockwise online softmax") cuts a sequence of
+ * S tokens into P shards of Sq = S/P tokens. Query shard i stays put; at ring step
+ * s = 0..P-1 it meets KV shard j = (i - s) mod P (section 2 "core principle";
+ * section 5 listing starts from the device's own block). Each block is folded into
+ * a running row state (m, l, O) by
+ *     S = Q_i K_j^T * scale,  m_new = max(m, rowmax S),  alpha = exp(m - m_new),
+ *     P = exp(S - m_new),     l = l*alpha + rowsum P,    O = O*alpha + P V_j,
+ * and the result is O / l. This equals ordinary softmax attention exactly (same
+ * section), so the output does not depend on P or on the layout; both select the
+ * order of the work. Causal masking (section 7 "causal attention with striped
+ * attention") lets query token t see keys u <= t (inclusive diagonal). Layout
+ * CONTIGUOUS puts tokens [i*Sq, (i+1)*Sq) on shard i; STRIPED puts token t on
+ * shard t mod P.
+ *
+ * Tensor layout (all row-major, contiguous, natural token order for both layouts):
+ *     q, out : [B, Hq,  S, D]      k, v : [B, Hkv, S, D]      lse : [B, Hq, S] fp32
+ * Query head h reads KV head h / (Hq/Hkv) (grouped-query attention when Hkv < Hq).
+ * lse = m + ln(l): natural log-sum-exp of the scaled scores of each row.
+ *
+ * Ownership. The caller allocates and frees every buffer (device memory unless
+ * stated). The library allocates no device memory and keeps no state between
+ * calls. All compute entry points are asynchronous on `stream` (a cudaStream_t
+ * passed as void*; NULL = legacy default stream); they return after enqueueing.
+ *
+ * Errors. Every entry point returns 0 on success or a negative RING_ATTN_E* code.
+ * On an argument error nothing is enqueued and no output is touched. A kernel
+ * whose internal wait exceeds its watchdog limit stops early, writes
+ * RING_ATTN_ETIMEOUT into the status word at the start of the workspace and
+ * leaves the outputs undefined; ring_attn_status() reports it.
+ */
+#ifndef RINGATTN_H_
+#define RINGATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define RING_ATTN_OK 0
+#define RING_ATTN_EINVAL (-1)       /* null pointer, non-positive size, S % P != 0, Hq % Hkv != 0, bad enum */
+#define RING_ATTN_EALIGN (-2)       /* a tensor pointer is not 16-byte aligned */
+#define RING_ATTN_EUNSUPPORTED (-3) /* D not in {64, 128}, or no sm_100 device for the tensor-core path */
+#define RING_ATTN_EWORKSPACE (-4)   /* workspace null or smaller than ring_attn_fwd_workspace_bytes() */
+#define RING_ATTN_ECUDA (-5)        /* a CUDA runtime/driver call failed (launch, tensor-map encode) */
+#define RING_ATTN_ETIMEOUT (-6)     /* a device-side wait hit its watchdog limit */
+
+#define RING_ATTN_LAYOUT_CONTIGUOUS 0
+#define RING_ATTN_LAYOUT_STRIPED 1
+
+#define RING_ATTN_DTYPE_FP32 0
+#define RING_ATTN_DTYPE_BF16 1
+
+#define RING_ATTN_ALGO_AUTO 0    /* bf16 -> tensor-core kernel, fp32 -> SIMT kernel */
+#define RING_ATTN_ALGO_SIMT 1    /* fp32-accumulating CUDA-core kernel (fp32 or bf16 inputs) */
+#define RING_ATTN_ALGO_TCGEN05 2 /* sm_100a tcgen05/TMEM/TMA kernel (bf16 inputs only) */
+
+/* Library version (major*10000 + minor*100 + patch). */
+int ring_attn_version(void);
+
+/* Text for an error code; never NULL. */
+const char* ring_attn_strerror(int code);
+
+/*
+ * Bytes of device workspace ring_attn_fwd needs for these arguments (>= 256:
+ * the first 4 bytes are the status word). Returns 0 for invalid arguments.
+ */
+size_t ring_attn_fwd_workspace_bytes(int B, int Hq, int Hkv, int64_t S, int D, int P,
+                                     int causal, int layout, int dtype);
+
+/*
+ * Exact attention over P ring shards: out = softmax(q k^T * scale, causal mask) v
+ * and lse, folding KV shards in ring order for every query shard.
+ *   q, k, v   device pointers, dtype `dtype`, shapes above, 16-byte aligned
+ *   out       device pointer [B,Hq,S,D] in `dtype` (bf16 rounded to nearest even)
+ *   lse       device pointer [B,Hq,S] fp32
+ *   S % P == 0, Hq % Hkv == 0, D in {64, 128}; causal 0|1; layout RING_ATTN_LAYOUT_*
+ *   scale     score scale (the pages use 1/sqrt(D))
+ *   workspace device scratch of >= ring_attn_fwd_workspace_bytes() bytes
+ * q/k/v must not alias out/lse.
+ */
+int ring_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
+                  int B, int Hq, int Hkv, int64_t S, int D, int P,
+                  int causal, int layout, float scale, int dtype,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* ring_attn_fwd with an explicit kernel choice (RING_ATTN_ALGO_*). */
+int ring_attn_fwd_algo(const void* q, const void* k, const void* v, void* out, float* lse,
+                       int B, int Hq, int Hkv, int64_t S, int D, int P,
+                       int causal, int layout, float scale, int dtype,
+                       void* workspace, size_t workspace_bytes, void* stream, int algo);
+
+/*
+ * One literal ring step: query shard i against KV shard j (any 0 <= i, j < P),
+ * as device i computes it at ring step (i - j) mod P. Writes the step's
+ * normalised partial in the shard's local order:
+ *   o_part   device [B, Hq, Sq, D] fp32 = softmax over the block's allowed keys, times V_j
+ *   lse_part device [B, Hq, Sq]    fp32, -inf for rows with no allowed key (then o_part row = 0)
+ * Merging the P steps of shard i with ring_attn_merge gives rows of ring_attn_fwd.
+ * Same argument rules as ring_attn_fwd; uses `workspace` for its status word.
+ */
+int ring_attn_fwd_step(const void* q, const void* k, const void* v, float* o_part, float* lse_part,
+                       int B, int Hq, int Hkv, int64_t S, int D, int P, int q_shard, int kv_shard,
+                       int causal, int layout, float scale, int dtype, int algo,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Combine n normalised partials of the same rows (the online-softmax rescale of
+ * section 3 applied to states whose l is already divided out):
+ *   lse = lse_max + ln sum_k exp(lse_k - lse_max),  out = sum_k exp(lse_k - lse) * o_k
+ *   o_parts   device [n_parts, rows, D] fp32     lse_parts device [n_parts, rows] fp32
+ *   out       device [rows, D] in out_dtype      lse_out   device [rows] fp32
+ * A part with lse_k = -inf is empty and its o_k is ignored; if all parts are
+ * empty the row gets out = 0, lse = -inf. D % 8 == 0, D <= 256. Outputs must
+ * not alias inputs. 1 <= n_parts <= 1024.
+ */
+int ring_attn_merge(const float* o_parts, const float* lse_parts, int n_parts, int64_t rows, int D,
+                    void* out, float* lse_out, int out_dtype, void* stream);
+
+/*
+ * Synchronise `stream` and read the status word at the start of `workspace`
+ * (written by the last compute call that used it): 0, or RING_ATTN_ETIMEOUT.
+ * Returns RING_ATTN_ECUDA if the stream reports an error.
+ */
+int ring_attn_status(const void* workspace, void* stream);
+
+/* ---- test hooks ------------------------------------------------------------ */
+
+/*
+ * Host only, no GPU. Walks the exact unit/tile schedule and per-element masks the
+ * kernels use (tile sizes tile_q x tile_k, any positive values) and adds 1 to
+ * counts[t*S + u] for every (query token t, key token u) pair the schedule lets
+ * into the softmax. counts is host memory of S*S int32, zeroed by the caller.
+ * S <= 4096. Returns the number of visited tiles (>= 0) or an error code.
+ */
+int64_t ring_attn_debug_visit_counts(int64_t S, int P, int causal, int layout,
+                                     int tile_q, int tile_k, int32_t* counts);
+
+/*
+ * Host only. Writes the fused kernel's work units in launch order for query
+ * blocks of tile_q rows: 5 int32 per unit (b, h, q_shard, row_block, kv tiles of
+ * 128 keys the unit visits). Returns the unit count, or an error code
+ * (RING_ATTN_EINVAL if it exceeds max_units).
+ */
+int ring_attn_debug_decode_units(int B, int Hq, int Hkv, int64_t S, int P, int causal, int layout, int tile_q,
+                                 int32_t* units_out, int64_t max_units);
+
+/*
+ * Host only. The (kv_shard, kv_tile) sequence, in visiting order, of work unit
+ * `unit` (launch order, query blocks of tile_q rows, key tiles of tile_k keys):
+ * 2 int32 per visited tile into pairs_out. Returns the tile count or an error
+ * code (RING_ATTN_EINVAL if it exceeds max_pairs or unit is out of range).
+ */
+int64_t ring_attn_debug_unit_walk(int B, int Hq, int Hkv, int64_t S, int P, int causal, int layout, int tile_q,
+                                  int tile_k, int64_t unit, int32_t* pairs_out, int64_t max_pairs);
+
+/*
+ * Host only. Fills info[0..5] for the fused-kernel grid of these arguments:
+ * number of units, total KV tiles visited, KV tiles with a partial mask, longest
+ * unit in tiles, first unit's tiles, last unit's tiles. Returns 0 or an error code.
+ */
+int ring_attn_debug_schedule_info(int B, int Hq, int Hkv, int64_t S, int D, int P,
+                                  int causal, int layout, int64_t* info);
+
+/*
+ * Launches one CTA that waits on an mbarrier nobody arrives on, with a watchdog
+ * limit of timeout_us microseconds; the wait gives up, the kernel records
+ * RING_ATTN_ETIMEOUT in the workspace status word and returns. Exercises the
+ * bounded-wait path without faulting or hanging the GPU.
+ */
+int ring_attn_debug_watchdog(int timeout_us, void* workspace, size_t workspace_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RINGATTN_H_ */

@@ -1,0 +1,12 @@
+"""Exact ring attention on one B200: C-ABI library (libringattn.so) + thin binding.
+
+The library (built in-tree by ``python -m sequence_exact_attention_ring_b200.build``)
+holds every kernel; this package only marshals arguments. Importing the package
+does not load the library; the first call does, and raises if it is missing.
+"""
+from . import binding  # noqa: F401
+from .api import HostRunner, merge, ring_attention, ring_attention_step, status, workspace_bytes  # noqa: F401
+from .binding import RingAttnError  # noqa: F401
+
+__all__ = ["binding", "ring_attention", "ring_attention_step", "merge", "status", "workspace_bytes",
+           "HostRunner", "RingAttnError"]

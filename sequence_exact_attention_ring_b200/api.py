@@ -1,0 +1,152 @@
+"""Torch-facing calls over the C ABI. PyTorch supplies device memory and streams.
+
+Marshalling only: shapes/dtypes are checked, buffers allocated with torch, and the
+library's kernels do every step of the computation.
+"""
+from __future__ import annotations
+
+import math
+
+import torch
+
+from . import binding as _b
+
+_LAYOUTS = {"contiguous": _b.LAYOUT_CONTIGUOUS, "striped": _b.LAYOUT_STRIPED}
+_ALGOS = {"auto": _b.ALGO_AUTO, "simt": _b.ALGO_SIMT, "tcgen05": _b.ALGO_TCGEN05}
+_DTYPES = {torch.float32: _b.DTYPE_FP32, torch.bfloat16: _b.DTYPE_BF16}
+
+
+def _stream_ptr(stream) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+def _layout(layout) -> int:
+    return _LAYOUTS[layout] if isinstance(layout, str) else int(layout)
+
+
+def _check_qkv(q, k, v):
+    if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
+        raise ValueError("q, k, v must be [B, H, S, D]")
+    if not (q.is_cuda and k.is_cuda and v.is_cuda):
+        raise ValueError("q, k, v must be CUDA tensors (use ring_attention_host for host buffers)")
+    if q.dtype not in _DTYPES or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must share dtype float32 or bfloat16")
+    if k.shape != v.shape or q.shape[0] != k.shape[0] or q.shape[2:] != k.shape[2:]:
+        raise ValueError("shape mismatch: q [B,Hq,S,D], k/v [B,Hkv,S,D]")
+    if not (q.is_contiguous() and k.is_contiguous() and v.is_contiguous()):
+        raise ValueError("q, k, v must be contiguous")
+
+
+def workspace_bytes(q: torch.Tensor, k: torch.Tensor, P: int, causal: bool, layout) -> int:
+    B, Hq, S, D = q.shape
+    n = _b.ring_attn_fwd_workspace_bytes(B, Hq, k.shape[1], S, D, P, int(causal), _layout(layout),
+                                         _DTYPES[q.dtype])
+    if n == 0:
+        raise _b.RingAttnError(_b.EINVAL, "ring_attn_fwd_workspace_bytes")
+    return n
+
+
+def ring_attention(q, k, v, P: int, causal: bool = True, layout="striped", scale: float | None = None,
+                   algo: str = "auto", out=None, lse=None, workspace=None, stream=None):
+    """Exact attention of q [B,Hq,S,D] over k/v [B,Hkv,S,D] folded in P ring shards.
+
+    Returns (out [B,Hq,S,D] in q's dtype, lse [B,Hq,S] fp32). Asynchronous on `stream`.
+    """
+    _check_qkv(q, k, v)
+    B, Hq, S, D = q.shape
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, S), dtype=torch.float32, device=q.device)
+    wsb = workspace_bytes(q, k, P, causal, layout)
+    if workspace is None:
+        workspace = torch.empty(wsb, dtype=torch.uint8, device=q.device)
+    rc = _b.ring_attn_fwd_algo(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                               B, Hq, k.shape[1], S, D, P, int(causal), _layout(layout), scale,
+                               _DTYPES[q.dtype], workspace.data_ptr(), workspace.numel(), _stream_ptr(stream),
+                               _ALGOS[algo])
+    _b.check(rc, "ring_attn_fwd")
+    return out, lse
+
+
+def ring_attention_step(q, k, v, P: int, q_shard: int, kv_shard: int, causal: bool = True, layout="striped",
+                        scale: float | None = None, algo: str = "auto", stream=None):
+    """One ring step: normalised partial (o [B,Hq,Sq,D] fp32, lse [B,Hq,Sq]) in shard-local order."""
+    _check_qkv(q, k, v)
+    B, Hq, S, D = q.shape
+    Sq = S // P
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    o = torch.empty((B, Hq, Sq, D), dtype=torch.float32, device=q.device)
+    lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    wsb = workspace_bytes(q, k, P, causal, layout)
+    ws = torch.empty(wsb, dtype=torch.uint8, device=q.device)
+    rc = _b.ring_attn_fwd_step(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, Hq,
+                               k.shape[1], S, D, P, q_shard, kv_shard, int(causal), _layout(layout), scale,
+                               _DTYPES[q.dtype], _ALGOS[algo], ws.data_ptr(), ws.numel(), _stream_ptr(stream))
+    _b.check(rc, "ring_attn_fwd_step")
+    return o, lse
+
+
+def merge(o_parts: torch.Tensor, lse_parts: torch.Tensor, out_dtype=torch.float32, stream=None):
+    """Merge normalised partials o_parts [n, ..., D] fp32 / lse_parts [n, ...] -> (out [..., D], lse [...])."""
+    if o_parts.dtype != torch.float32 or lse_parts.dtype != torch.float32:
+        raise ValueError("partials must be float32")
+    if not (o_parts.is_cuda and lse_parts.is_cuda and o_parts.is_contiguous() and lse_parts.is_contiguous()):
+        raise ValueError("partials must be contiguous CUDA tensors")
+    n, D = o_parts.shape[0], o_parts.shape[-1]
+    lead = o_parts.shape[1:-1]
+    if tuple(lse_parts.shape) != (n, *lead):
+        raise ValueError("lse_parts must be [n, ...] matching o_parts [n, ..., D]")
+    rows = int(math.prod(lead))
+    out = torch.empty((*lead, D), dtype=out_dtype, device=o_parts.device)
+    lse = torch.empty(lead, dtype=torch.float32, device=o_parts.device)
+    rc = _b.ring_attn_merge(o_parts.data_ptr(), lse_parts.data_ptr(), n, rows, D, out.data_ptr(), lse.data_ptr(),
+                            _DTYPES[out_dtype], _stream_ptr(stream))
+    _b.check(rc, "ring_attn_merge")
+    return out, lse
+
+
+def status(workspace: torch.Tensor, stream=None) -> int:
+    """Synchronise and return the workspace status word (0 or binding.ETIMEOUT)."""
+    return _b.ring_attn_status(workspace.data_ptr(), _stream_ptr(stream))
+
+
+class HostRunner:
+    """End-to-end path for host-resident inputs: pinned host -> device copies,
+    ring_attn_fwd, device -> pinned host copies, all on one stream.
+
+    Device buffers are allocated once (by torch) and reused across calls.
+    """
+
+    def __init__(self, shape_q, shape_kv, dtype, P, causal=True, layout="striped", scale=None, device="cuda"):
+        self.P, self.causal, self.layout = P, causal, layout
+        B, Hq, S, D = shape_q
+        self.scale = 1.0 / math.sqrt(D) if scale is None else scale
+        self.q = torch.empty(shape_q, dtype=dtype, device=device)
+        self.k = torch.empty(shape_kv, dtype=dtype, device=device)
+        self.v = torch.empty(shape_kv, dtype=dtype, device=device)
+        self.out = torch.empty(shape_q, dtype=dtype, device=device)
+        self.lse = torch.empty((B, Hq, S), dtype=torch.float32, device=device)
+        self.out_host = torch.empty(shape_q, dtype=dtype, pin_memory=True)
+        self.lse_host = torch.empty((B, Hq, S), dtype=torch.float32, pin_memory=True)
+        self.ws = torch.empty(workspace_bytes(self.q, self.k, P, causal, layout), dtype=torch.uint8, device=device)
+
+    def h2d_bytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in (self.q, self.k, self.v))
+
+    def d2h_bytes(self) -> int:
+        return self.out.numel() * self.out.element_size() + self.lse.numel() * 4
+
+    def run(self, q_host, k_host, v_host, stream=None):
+        s = stream if stream is not None else torch.cuda.current_stream()
+        with torch.cuda.stream(s):
+            self.q.copy_(q_host, non_blocking=True)
+            self.k.copy_(k_host, non_blocking=True)
+            self.v.copy_(v_host, non_blocking=True)
+            ring_attention(self.q, self.k, self.v, self.P, self.causal, self.layout, self.scale, out=self.out,
+                           lse=self.lse, workspace=self.ws, stream=s)
+            self.out_host.copy_(self.out, non_blocking=True)
+            self.lse_host.copy_(self.lse, non_blocking=True)
+        return self.out_host, self.lse_host

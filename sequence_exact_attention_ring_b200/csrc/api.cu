@@ -1,0 +1,312 @@
+// C ABI of libringattn.so: argument validation, dispatch, status word, test hooks.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include "../../include/ringattn.h"
+#include "ring_schedule.h"
+#include "ringattn_internal.h"
+#include "sm100_ptx.cuh"
+
+using namespace ringattn;
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_geom(int B, int Hq, int Hkv, int64_t S, int D, int P, int causal, int layout, int dtype, RingGeom* g) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || S <= 0 || D <= 0 || P <= 0) return RING_ATTN_EINVAL;
+  if (S % P != 0 || Hq % Hkv != 0) return RING_ATTN_EINVAL;
+  if (causal != 0 && causal != 1) return RING_ATTN_EINVAL;
+  if (layout != RING_ATTN_LAYOUT_CONTIGUOUS && layout != RING_ATTN_LAYOUT_STRIPED) return RING_ATTN_EINVAL;
+  if (dtype != RING_ATTN_DTYPE_FP32 && dtype != RING_ATTN_DTYPE_BF16) return RING_ATTN_EINVAL;
+  if ((int64_t)B * Hq > (1 << 24) || S > ((int64_t)1 << 31)) return RING_ATTN_EINVAL;
+  if (D != 64 && D != 128) return RING_ATTN_EUNSUPPORTED;
+  g->B = B;
+  g->Hq = Hq;
+  g->Hkv = Hkv;
+  g->S = S;
+  g->D = D;
+  g->P = P;
+  g->causal = causal;
+  g->layout = layout;
+  g->Sq = S / P;
+  return RING_ATTN_OK;
+}
+
+// sm_100 family check for the tensor-core path, cached per device ordinal.
+bool device_is_sm100() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  static int cache[64];  // 0 unknown, 1 yes, 2 no
+  if (dev < 0 || dev >= 64) return false;
+  if (cache[dev] == 0) {
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    cache[dev] = (major == 10 && minor == 0) ? 1 : 2;
+  }
+  return cache[dev] == 1;
+}
+
+uint64_t watchdog_ns() {
+  static uint64_t ns = 0;
+  if (ns == 0) {
+    uint64_t ms = 2000;
+    const char* e = getenv("RING_ATTN_WATCHDOG_MS");
+    if (e && atoi(e) > 0) ms = (uint64_t)atoi(e);
+    ns = ms * 1000000ull;
+  }
+  return ns;
+}
+
+int resolve_algo(int algo, int dtype) {
+  if (algo == RING_ATTN_ALGO_AUTO) return dtype == RING_ATTN_DTYPE_BF16 ? RING_ATTN_ALGO_TCGEN05 : RING_ATTN_ALGO_SIMT;
+  return algo;
+}
+
+int check_algo(int algo, int dtype) {
+  if (algo != RING_ATTN_ALGO_SIMT && algo != RING_ATTN_ALGO_TCGEN05) return RING_ATTN_EINVAL;
+  if (algo == RING_ATTN_ALGO_TCGEN05 && (dtype != RING_ATTN_DTYPE_BF16 || !device_is_sm100()))
+    return RING_ATTN_EUNSUPPORTED;
+  return RING_ATTN_OK;
+}
+
+int reset_status(void* workspace, cudaStream_t stream) {
+  return cudaMemsetAsync(workspace, 0, sizeof(int), stream) == cudaSuccess ? RING_ATTN_OK : RING_ATTN_ECUDA;
+}
+
+// Launch one ring-attention pass for the given ring-step range and output mode.
+int run_fwd(const void* q, const void* k, const void* v, void* out, float* lse, const RingGeom& g, float scale,
+            int dtype, int algo, int s_begin, int s_end, int q_shard_only, int partial, void* workspace,
+            cudaStream_t stream) {
+  int rc = reset_status(workspace, stream);
+  if (rc) return rc;
+  if (algo == RING_ATTN_ALGO_TCGEN05)
+    return launch_fwd_sm100(q, k, v, out, lse, g, scale, s_begin, s_end, q_shard_only, partial,
+                            static_cast<int*>(workspace), watchdog_ns(), stream);
+  return launch_fwd_simt(q, k, v, out, lse, g, scale, dtype, s_begin, s_end, q_shard_only, partial, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+int ring_attn_version(void) { return kVersion; }
+
+const char* ring_attn_strerror(int code) {
+  switch (code) {
+    case RING_ATTN_OK: return "success";
+    case RING_ATTN_EINVAL: return "invalid argument";
+    case RING_ATTN_EALIGN: return "pointer not 16-byte aligned";
+    case RING_ATTN_EUNSUPPORTED: return "unsupported configuration (head dim, dtype or device)";
+    case RING_ATTN_EWORKSPACE: return "workspace missing or too small";
+    case RING_ATTN_ECUDA: return "CUDA call failed";
+    case RING_ATTN_ETIMEOUT: return "device wait exceeded its watchdog limit";
+    default: return "unknown error";
+  }
+}
+
+size_t ring_attn_fwd_workspace_bytes(int B, int Hq, int Hkv, int64_t S, int D, int P, int causal, int layout,
+                                     int dtype) {
+  RingGeom g;
+  if (check_geom(B, Hq, Hkv, S, D, P, causal, layout, dtype, &g) != RING_ATTN_OK) return 0;
+  return kWorkspaceHeaderBytes;
+}
+
+int ring_attn_fwd_algo(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv,
+                       int64_t S, int D, int P, int causal, int layout, float scale, int dtype, void* workspace,
+                       size_t workspace_bytes, void* stream, int algo) {
+  RingGeom g;
+  int rc = check_geom(B, Hq, Hkv, S, D, P, causal, layout, dtype, &g);
+  if (rc) return rc;
+  if (!q || !k || !v || !out || !lse) return RING_ATTN_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+    return RING_ATTN_EALIGN;
+  if (!workspace || workspace_bytes < kWorkspaceHeaderBytes || !aligned16(workspace)) return RING_ATTN_EWORKSPACE;
+  algo = resolve_algo(algo, dtype);
+  if ((rc = check_algo(algo, dtype))) return rc;
+  return run_fwd(q, k, v, out, lse, g, scale, dtype, algo, 0, P, -1, 0, workspace,
+                 static_cast<cudaStream_t>(stream));
+}
+
+int ring_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv,
+                  int64_t S, int D, int P, int causal, int layout, float scale, int dtype, void* workspace,
+                  size_t workspace_bytes, void* stream) {
+  return ring_attn_fwd_algo(q, k, v, out, lse, B, Hq, Hkv, S, D, P, causal, layout, scale, dtype, workspace,
+                            workspace_bytes, stream, RING_ATTN_ALGO_AUTO);
+}
+
+int ring_attn_fwd_step(const void* q, const void* k, const void* v, float* o_part, float* lse_part, int B, int Hq,
+                       int Hkv, int64_t S, int D, int P, int q_shard, int kv_shard, int causal, int layout,
+                       float scale, int dtype, int algo, void* workspace, size_t workspace_bytes, void* stream) {
+  RingGeom g;
+  int rc = check_geom(B, Hq, Hkv, S, D, P, causal, layout, dtype, &g);
+  if (rc) return rc;
+  if (q_shard < 0 || q_shard >= P || kv_shard < 0 || kv_shard >= P) return RING_ATTN_EINVAL;
+  if (!q || !k || !v || !o_part || !lse_part) return RING_ATTN_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o_part) || !aligned16(lse_part))
+    return RING_ATTN_EALIGN;
+  if (!workspace || workspace_bytes < kWorkspaceHeaderBytes || !aligned16(workspace)) return RING_ATTN_EWORKSPACE;
+  algo = resolve_algo(algo, dtype);
+  if ((rc = check_algo(algo, dtype))) return rc;
+  const int s = ring_step_of(q_shard, kv_shard, P);
+  return run_fwd(q, k, v, o_part, lse_part, g, scale, dtype, algo, s, s + 1, q_shard, 1, workspace,
+                 static_cast<cudaStream_t>(stream));
+}
+
+int ring_attn_merge(const float* o_parts, const float* lse_parts, int n_parts, int64_t rows, int D, void* out,
+                    float* lse_out, int out_dtype, void* stream) {
+  if (!o_parts || !lse_parts || !out || !lse_out) return RING_ATTN_EINVAL;
+  if (n_parts < 1 || n_parts > 1024 || rows < 0 || D <= 0 || D % 8 != 0 || D > 256) return RING_ATTN_EINVAL;
+  if (out_dtype != RING_ATTN_DTYPE_FP32 && out_dtype != RING_ATTN_DTYPE_BF16) return RING_ATTN_EINVAL;
+  if (!aligned16(o_parts) || !aligned16(out) || !aligned16(lse_parts) || !aligned16(lse_out)) return RING_ATTN_EALIGN;
+  return launch_merge(o_parts, lse_parts, n_parts, rows, D, out, lse_out, out_dtype,
+                      static_cast<cudaStream_t>(stream));
+}
+
+int ring_attn_status(const void* workspace, void* stream) {
+  if (!workspace) return RING_ATTN_EINVAL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return RING_ATTN_ECUDA;
+  int status = 0;
+  if (cudaMemcpy(&status, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return RING_ATTN_ECUDA;
+  return status;
+}
+
+int64_t ring_attn_debug_visit_counts(int64_t S, int P, int causal, int layout, int tile_q, int tile_k,
+                                     int32_t* counts) {
+  RingGeom g;
+  int rc = check_geom(1, 1, 1, S, 64, P, causal, layout, RING_ATTN_DTYPE_BF16, &g);
+  if (rc) return rc;
+  if (!counts || tile_q <= 0 || tile_k <= 0 || S > 4096) return RING_ATTN_EINVAL;
+  int64_t tiles = 0;
+  const int64_t units = num_units(g, tile_q, -1);
+  for (int64_t u = 0; u < units; ++u) {
+    const Unit U = decode_unit(g, tile_q, -1, u);
+    const int64_t a0 = (int64_t)U.tb * tile_q;
+    const int64_t a_hi = (a0 + tile_q - 1 < g.Sq - 1) ? a0 + tile_q - 1 : g.Sq - 1;
+    for (TileWalk w = walk_begin(g, U.i, a_hi, tile_k, 0, P); walk_valid(w); walk_next(g, w, a_hi, tile_k)) {
+      ++tiles;
+      for (int64_t a = a0; a < a0 + tile_q && a < g.Sq; ++a) {
+        const int64_t lim = key_limit(g, U.i, w.j, a);
+        for (int c = 0; c < tile_k; ++c) {
+          const int64_t b = (int64_t)w.kb * tile_k + c;
+          if (b < lim) counts[token_of(g, U.i, a) * S + token_of(g, w.j, b)] += 1;
+        }
+      }
+    }
+  }
+  return tiles;
+}
+
+int ring_attn_debug_decode_units(int B, int Hq, int Hkv, int64_t S, int P, int causal, int layout, int tile_q,
+                                 int32_t* units_out, int64_t max_units) {
+  RingGeom g;
+  int rc = check_geom(B, Hq, Hkv, S, 64, P, causal, layout, RING_ATTN_DTYPE_BF16, &g);
+  if (rc) return rc;
+  if (tile_q <= 0) return RING_ATTN_EINVAL;
+  const int64_t n = num_units(g, tile_q, -1);
+  if (!units_out || n > max_units) return RING_ATTN_EINVAL;
+  for (int64_t u = 0; u < n; ++u) {
+    const Unit U = decode_unit(g, tile_q, -1, u);
+    const int64_t a0 = (int64_t)U.tb * tile_q;
+    const int64_t a_hi = (a0 + tile_q - 1 < g.Sq - 1) ? a0 + tile_q - 1 : g.Sq - 1;
+    units_out[5 * u + 0] = U.b;
+    units_out[5 * u + 1] = U.h;
+    units_out[5 * u + 2] = U.i;
+    units_out[5 * u + 3] = U.tb;
+    units_out[5 * u + 4] = (int32_t)unit_tile_count(g, U.i, a_hi, 128, 0, P);
+  }
+  return (int)n;
+}
+
+int64_t ring_attn_debug_unit_walk(int B, int Hq, int Hkv, int64_t S, int P, int causal, int layout, int tile_q,
+                                  int tile_k, int64_t unit, int32_t* pairs_out, int64_t max_pairs) {
+  RingGeom g;
+  int rc = check_geom(B, Hq, Hkv, S, 64, P, causal, layout, RING_ATTN_DTYPE_BF16, &g);
+  if (rc) return rc;
+  if (tile_q <= 0 || tile_k <= 0 || !pairs_out || unit < 0 || unit >= num_units(g, tile_q, -1))
+    return RING_ATTN_EINVAL;
+  const Unit U = decode_unit(g, tile_q, -1, unit);
+  const int64_t a0 = (int64_t)U.tb * tile_q;
+  const int64_t a_hi = (a0 + tile_q - 1 < g.Sq - 1) ? a0 + tile_q - 1 : g.Sq - 1;
+  int64_t n = 0;
+  for (TileWalk w = walk_begin(g, U.i, a_hi, tile_k, 0, P); walk_valid(w); walk_next(g, w, a_hi, tile_k), ++n) {
+    if (n >= max_pairs) return RING_ATTN_EINVAL;
+    pairs_out[2 * n] = w.j;
+    pairs_out[2 * n + 1] = w.kb;
+  }
+  return n;
+}
+
+int ring_attn_debug_schedule_info(int B, int Hq, int Hkv, int64_t S, int D, int P, int causal, int layout,
+                                  int64_t* info) {
+  RingGeom g;
+  int rc = check_geom(B, Hq, Hkv, S, D, P, causal, layout, RING_ATTN_DTYPE_BF16, &g);
+  if (rc) return rc;
+  if (!info) return RING_ATTN_EINVAL;
+  const int BQ = 256, BN = 128;
+  const int64_t units = num_units(g, BQ, -1);
+  int64_t total = 0, partial = 0, longest = 0, first = 0, last = 0;
+  for (int64_t u = 0; u < units; ++u) {
+    const Unit U = decode_unit(g, BQ, -1, u);
+    const int64_t a0 = (int64_t)U.tb * BQ;
+    const int64_t a_hi = (a0 + BQ - 1 < g.Sq - 1) ? a0 + BQ - 1 : g.Sq - 1;
+    int64_t n = 0;
+    for (TileWalk w = walk_begin(g, U.i, a_hi, BN, 0, P); walk_valid(w); walk_next(g, w, a_hi, BN)) {
+      ++n;
+      if ((int64_t)w.kb * BN + BN > key_limit(g, U.i, w.j, a0)) ++partial;
+    }
+    total += n;
+    if (n > longest) longest = n;
+    if (u == 0) first = n;
+    last = n;
+  }
+  info[0] = units;
+  info[1] = total;
+  info[2] = partial;
+  info[3] = longest;
+  info[4] = first;
+  info[5] = last;
+  return RING_ATTN_OK;
+}
+
+int ring_attn_debug_watchdog(int timeout_us, void* workspace, size_t workspace_bytes, void* stream) {
+  if (timeout_us <= 0 || timeout_us > 10000000) return RING_ATTN_EINVAL;
+  if (!workspace || workspace_bytes < kWorkspaceHeaderBytes) return RING_ATTN_EWORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int rc = reset_status(workspace, s);
+  if (rc) return rc;
+  return launch_watchdog_probe(timeout_us, static_cast<int*>(workspace), s);
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- watchdog probe
+namespace ringattn {
+
+__global__ void watchdog_probe_kernel(int* status, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+  const Watchdog wd{&abort_flag, status, limit_ns};
+  // nobody arrives on `bar`: the bounded wait must give up and report
+  (void)mbar_wait(&bar, 0, wd);
+  __syncthreads();
+}
+
+int launch_watchdog_probe(int timeout_us, int* status, cudaStream_t stream) {
+  watchdog_probe_kernel<<<1, 32, 0, stream>>>(status, (uint64_t)timeout_us * 1000ull);
+  return cudaGetLastError() == cudaSuccess ? RING_ATTN_OK : RING_ATTN_ECUDA;
+}
+
+}  // namespace ringattn

@@ -1,0 +1,99 @@
+// Merge of normalised partial attention results (HBM-bound, vectorised).
+//
+// A partial k covers a subset of the keys of a row and holds O_k = (its softmax
+// weights) * V and lse_k = ln(sum of its exponentials). The online-softmax rescale
+// of the RingAttention deep-architecture article (techknowgenie), section 3
+// (alpha = exp(m_old - m_new), beta = exp(m_block - m_new)) applied to such
+// normalised states gives
+//     lse = lse_max + ln sum_k exp(lse_k - lse_max),   O = sum_k exp(lse_k - lse) O_k.
+// Empty partials (lse_k = -inf) get weight 0; an all-empty row yields O = 0, lse = -inf.
+//
+// Each thread owns 8 consecutive columns of one row: two 16-byte fp32 loads per
+// partial, one 16-byte bf16 store (or two fp32 stores) per row chunk.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "ringattn_internal.h"
+
+namespace ringattn {
+namespace merge {
+
+constexpr int kThreads = 256;
+constexpr int kVec = 8;
+
+template <bool kBf16Out>
+__global__ void __launch_bounds__(kThreads) merge_kernel(const float* __restrict__ o_parts,
+                                                         const float* __restrict__ lse_parts, int n_parts,
+                                                         int64_t rows, int D, void* __restrict__ out,
+                                                         float* __restrict__ lse_out) {
+  const int tpr = D / kVec;  // threads per row
+  const int rows_per_block = kThreads / tpr;
+  const int64_t row = (int64_t)blockIdx.x * rows_per_block + threadIdx.x / tpr;
+  const int col = (threadIdx.x % tpr) * kVec;
+  if (threadIdx.x >= rows_per_block * tpr || row >= rows) return;
+
+  float mx = -INFINITY;
+  for (int k = 0; k < n_parts; ++k) mx = fmaxf(mx, __ldg(lse_parts + (int64_t)k * rows + row));
+  float acc[kVec];
+#pragma unroll
+  for (int e = 0; e < kVec; ++e) acc[e] = 0.f;
+  float lse_v = -INFINITY;
+  if (mx != -INFINITY) {
+    float tot = 0.f;
+    for (int k = 0; k < n_parts; ++k) {
+      const float lk = __ldg(lse_parts + (int64_t)k * rows + row);
+      if (lk == -INFINITY) continue;
+      const float wk = expf(lk - mx);
+      tot += wk;
+      const float4* src = reinterpret_cast<const float4*>(o_parts + ((int64_t)k * rows + row) * D + col);
+      const float4 x0 = __ldg(src);
+      const float4 x1 = __ldg(src + 1);
+      acc[0] = fmaf(wk, x0.x, acc[0]);
+      acc[1] = fmaf(wk, x0.y, acc[1]);
+      acc[2] = fmaf(wk, x0.z, acc[2]);
+      acc[3] = fmaf(wk, x0.w, acc[3]);
+      acc[4] = fmaf(wk, x1.x, acc[4]);
+      acc[5] = fmaf(wk, x1.y, acc[5]);
+      acc[6] = fmaf(wk, x1.z, acc[6]);
+      acc[7] = fmaf(wk, x1.w, acc[7]);
+    }
+    const float inv = 1.f / tot;
+#pragma unroll
+    for (int e = 0; e < kVec; ++e) acc[e] *= inv;
+    lse_v = mx + logf(tot);
+  }
+  if (kBf16Out) {
+    __nv_bfloat162 h[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) h[e] = __floats2bfloat162_rn(acc[2 * e], acc[2 * e + 1]);
+    *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(out) + row * D + col) =
+        *reinterpret_cast<const uint4*>(h);
+  } else {
+    float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + row * D + col);
+    dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+  }
+  if (threadIdx.x % tpr == 0) lse_out[row] = lse_v;
+}
+
+}  // namespace merge
+
+int launch_merge(const float* o_parts, const float* lse_parts, int n_parts, int64_t rows, int D, void* out,
+                 float* lse_out, int out_dtype, cudaStream_t stream) {
+  if (rows == 0) return RING_ATTN_OK;
+  const int tpr = D / merge::kVec;
+  const int rows_per_block = merge::kThreads / tpr;
+  const int64_t blocks = (rows + rows_per_block - 1) / rows_per_block;
+  if (blocks > 0x7fffffff) return RING_ATTN_EINVAL;
+  if (out_dtype == RING_ATTN_DTYPE_BF16)
+    merge::merge_kernel<true><<<(unsigned)blocks, merge::kThreads, 0, stream>>>(o_parts, lse_parts, n_parts, rows,
+                                                                                 D, out, lse_out);
+  else
+    merge::merge_kernel<false><<<(unsigned)blocks, merge::kThreads, 0, stream>>>(o_parts, lse_parts, n_parts,
+                                                                                  rows, D, out, lse_out);
+  return cudaGetLastError() == cudaSuccess ? RING_ATTN_OK : RING_ATTN_ECUDA;
+}
+
+}  // namespace ringattn

@@ -1,0 +1,169 @@
+// Ring geometry and schedule shared by the host scheduler and every kernel.
+//
+// RingAttention deep-architecture article (techknowgenie):
+//   section 2 "core principle": the sequence of S tokens is cut into P shards of
+//     Sq = S/P tokens; query shard i never moves, and at ring step s it meets the
+//     KV shard (i - s) mod P (blocks travel to the next device, arrive from the
+//     previous one; step 0 is the device's own block, per the section 5 listing).
+//   section 7 "causal attention with striped attention": under a causal mask
+//     token t sees only tokens u <= t (inclusive diagonal); the striped layout
+//     deals tokens round-robin, token t on shard t mod P.
+//
+// On one GPU the ring becomes the order in which a work unit visits KV tiles.
+// Everything here is plain integer arithmetic, compiled for both host and device
+// so the CPU tests check the exact code the kernels run.
+#pragma once
+
+#include <stdint.h>
+
+#if defined(__CUDACC__)
+#define RA_HD __host__ __device__ __forceinline__
+#else
+#define RA_HD inline
+#endif
+
+namespace ringattn {
+
+enum Layout : int { kContiguous = 0, kStriped = 1 };
+
+struct RingGeom {
+  int B, Hq, Hkv;
+  int64_t S;
+  int D, P;
+  int causal;   // 0 | 1
+  int layout;   // kContiguous | kStriped
+  int64_t Sq;   // S / P
+};
+
+// Global token of local index a in shard i.
+//   contiguous: shard i = tokens [i*Sq, (i+1)*Sq); striped: token a*P + i.
+RA_HD int64_t token_of(const RingGeom& g, int i, int64_t a) {
+  return g.layout == kStriped ? a * g.P + i : (int64_t)i * g.Sq + a;
+}
+
+// KV shard met by query shard i at ring step s (0 <= s < P).
+RA_HD int ring_kv_shard(int i, int s, int P) { return (i - s + P) % P; }
+
+// Ring step at which query shard i meets KV shard j.
+RA_HD int ring_step_of(int i, int j, int P) { return (i - j + P) % P; }
+
+// Keys of shard j visible to the query with local index a in shard i are exactly
+// the local indices b < key_limit(g, i, j, a) (always further capped at Sq).
+//   contiguous causal: j < i all keys; j == i keys b <= a; j > i none.
+//   striped causal: token b*P+j <= a*P+i  <=>  b < a, or b == a and j <= i.
+RA_HD int64_t key_limit(const RingGeom& g, int i, int j, int64_t a) {
+  int64_t lim;
+  if (!g.causal) {
+    lim = g.Sq;
+  } else if (g.layout == kContiguous) {
+    lim = (j < i) ? g.Sq : (j == i ? a + 1 : 0);
+  } else {
+    lim = (j <= i) ? a + 1 : a;
+  }
+  return lim < g.Sq ? lim : g.Sq;
+}
+
+// Number of TK-key tiles of shard j that the query rows [.., a_hi] of shard i
+// must visit (key_limit is non-decreasing in a, so the last row decides).
+RA_HD int kv_tiles_for(const RingGeom& g, int i, int j, int64_t a_hi, int TK) {
+  int64_t lim = key_limit(g, i, j, a_hi);
+  return (int)((lim + TK - 1) / TK);
+}
+
+// Work units. A unit is (b, h, q shard i, block of BQ query rows tb), folding
+// ring steps [s_begin, s_end). Units are numbered longest-first so that a grid
+// launched in index order approximates longest-processing-time scheduling:
+//   contiguous causal: cost grows with i*nkt + (rows of tb), so order by the
+//     combined index c = i*nblk + tb, descending;
+//   otherwise (striped causal, non-causal): cost depends on tb only, so order by
+//     tb descending; inside a tb the unit index runs over (b, kv head, i, head in
+//     the GQA group) so concurrently running units share K/V through L2.
+struct Unit {
+  int b, h, i, tb;
+};
+
+RA_HD int64_t num_row_blocks(const RingGeom& g, int BQ) { return (g.Sq + BQ - 1) / BQ; }
+
+RA_HD int64_t num_units(const RingGeom& g, int BQ, int q_shard_only) {
+  int64_t shards = q_shard_only >= 0 ? 1 : g.P;
+  return (int64_t)g.B * g.Hq * shards * num_row_blocks(g, BQ);
+}
+
+RA_HD Unit decode_unit(const RingGeom& g, int BQ, int q_shard_only, int64_t u) {
+  const int64_t nblk = num_row_blocks(g, BQ);
+  const int rep = g.Hq / g.Hkv;
+  Unit r;
+  if (q_shard_only >= 0) {
+    // a single query shard (one literal ring step): (tb desc, b, head)
+    const int64_t bh_n = (int64_t)g.B * g.Hq;
+    r.tb = (int)(nblk - 1 - u / bh_n);
+    int64_t bh = u % bh_n;
+    r.b = (int)(bh / g.Hq);
+    r.h = (int)(bh % g.Hq);
+    r.i = q_shard_only;
+    return r;
+  }
+  if (g.causal && g.layout == kContiguous) {
+    const int64_t bh_n = (int64_t)g.B * g.Hq;
+    const int64_t c = (int64_t)g.P * nblk - 1 - u / bh_n;
+    int64_t bh = u % bh_n;
+    r.i = (int)(c / nblk);
+    r.tb = (int)(c % nblk);
+    int64_t bg = bh / rep;  // (b, kv head) outer, GQA group member inner
+    r.b = (int)(bg / g.Hkv);
+    r.h = (int)((bg % g.Hkv) * rep + bh % rep);
+    return r;
+  }
+  const int64_t per_tb = (int64_t)g.B * g.Hq * g.P;
+  r.tb = (int)(nblk - 1 - u / per_tb);
+  int64_t x = u % per_tb;             // ((b*Hkv + kvh)*P + i)*rep + hr
+  const int hr = (int)(x % rep);
+  x /= rep;
+  r.i = (int)(x % g.P);
+  x /= g.P;
+  const int kvh = (int)(x % g.Hkv);
+  r.b = (int)(x / g.Hkv);
+  r.h = kvh * rep + hr;
+  return r;
+}
+
+// Total KV tiles a unit visits over ring steps [s_begin, s_end).
+RA_HD int64_t unit_tile_count(const RingGeom& g, int i, int64_t a_hi, int TK, int s_begin, int s_end) {
+  int64_t n = 0;
+  for (int s = s_begin; s < s_end; ++s) n += kv_tiles_for(g, i, ring_kv_shard(i, s, g.P), a_hi, TK);
+  return n;
+}
+
+// Incremental walk over the (ring step, kv tile) sequence of one unit; every role
+// of a kernel advances an identical copy, so they agree on every tile.
+struct TileWalk {
+  int s, s_end, j, kb, nkb;
+  int i, P;
+};
+
+RA_HD void walk_skip_empty(const RingGeom& g, TileWalk& w, int64_t a_hi, int TK) {
+  while (w.s < w.s_end) {
+    w.j = ring_kv_shard(w.i, w.s, g.P);
+    w.nkb = kv_tiles_for(g, w.i, w.j, a_hi, TK);
+    if (w.nkb > 0) return;
+    ++w.s;
+  }
+}
+
+RA_HD TileWalk walk_begin(const RingGeom& g, int i, int64_t a_hi, int TK, int s_begin, int s_end) {
+  TileWalk w;
+  w.s = s_begin; w.s_end = s_end; w.i = i; w.P = g.P; w.kb = 0; w.j = 0; w.nkb = 0;
+  walk_skip_empty(g, w, a_hi, TK);
+  return w;
+}
+
+RA_HD bool walk_valid(const TileWalk& w) { return w.s < w.s_end; }
+
+RA_HD void walk_next(const RingGeom& g, TileWalk& w, int64_t a_hi, int TK) {
+  if (++w.kb < w.nkb) return;
+  w.kb = 0;
+  ++w.s;
+  walk_skip_empty(g, w, a_hi, TK);
+}
+
+}  // namespace ringattn

@@ -1,0 +1,37 @@
+// Internal declarations shared by the C-ABI layer and the kernel files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/ringattn.h"
+#include "ring_schedule.h"
+
+namespace ringattn {
+
+typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// Status word layout at the start of the caller's workspace.
+constexpr size_t kWorkspaceHeaderBytes = 256;
+
+// Fused tcgen05 kernel (bf16). partial=0: final bf16 output in natural token order;
+// partial=1: normalised fp32 per-step partial in shard-local order.
+int launch_fwd_sm100(const void* q, const void* k, const void* v, void* out, float* lse, const RingGeom& g,
+                     float scale, int s_begin, int s_end, int q_shard_only, int partial, int* status,
+                     uint64_t watchdog_ns, cudaStream_t stream);
+int64_t fwd_sm100_units(const RingGeom& g, int q_shard_only);
+
+// fp32-accumulating SIMT kernel (fp32 or bf16 inputs), same schedule and output modes.
+int launch_fwd_simt(const void* q, const void* k, const void* v, void* out, float* lse, const RingGeom& g,
+                    float scale, int dtype, int s_begin, int s_end, int q_shard_only, int partial,
+                    cudaStream_t stream);
+
+int launch_merge(const float* o_parts, const float* lse_parts, int n_parts, int64_t rows, int D, void* out,
+                 float* lse_out, int out_dtype, cudaStream_t stream);
+
+int launch_watchdog_probe(int timeout_us, int* status, cudaStream_t stream);
+
+}  // namespace ringattn

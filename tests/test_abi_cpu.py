@@ -1,0 +1,184 @@
+"""The C-ABI library on the host: symbols, argument errors, the exact schedule.
+
+No compute call is made here (no GPU in this environment); every check runs on
+host code paths that return before touching CUDA.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle
+from sequence_exact_attention_ring_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ringattn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from sequence_exact_attention_ring_b200 import build
+    build.build()
+    return B.load()
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ring_attn_\w+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = header_functions()
+    assert len(names) >= 10
+    nm = subprocess.run(["nm", "-D", "--defined-only", B.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (ring_attn_\w+)", nm))
+    for n in names:
+        assert n in exported, n
+        assert hasattr(lib, n)
+        assert n in B.SIGNATURES, f"binding lacks {n}"
+
+
+def test_version_and_strerror(lib):
+    assert B.ring_attn_version() >= 100
+    for code in (B.OK, B.EINVAL, B.EALIGN, B.EUNSUPPORTED, B.EWORKSPACE, B.ECUDA, B.ETIMEOUT):
+        assert B.strerror(code) != "unknown error"
+    assert B.strerror(-99) == "unknown error"
+
+
+GOOD = dict(B=1, Hq=4, Hkv=2, S=1024, D=128, P=4, causal=1, layout=1, dtype=1)
+FAKE = 0x10000  # aligned, never dereferenced: every call below fails validation first
+
+
+def fwd(**kw):
+    a = dict(GOOD)
+    ptrs = dict(q=FAKE, k=FAKE, v=FAKE, out=FAKE, lse=FAKE, ws=FAKE, wsb=256)
+    for key in list(kw):
+        if key in ptrs:
+            ptrs[key] = kw.pop(key)
+    a.update(kw)
+    return B.ring_attn_fwd(ptrs["q"], ptrs["k"], ptrs["v"], ptrs["out"], ptrs["lse"], a["B"], a["Hq"], a["Hkv"],
+                           a["S"], a["D"], a["P"], a["causal"], a["layout"], 0.1, a["dtype"], ptrs["ws"],
+                           ptrs["wsb"], None)
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(B=0), B.EINVAL), (dict(Hq=0), B.EINVAL), (dict(S=0), B.EINVAL), (dict(P=0), B.EINVAL),
+    (dict(S=1000, P=3), B.EINVAL), (dict(Hq=3, Hkv=2), B.EINVAL), (dict(causal=2), B.EINVAL),
+    (dict(layout=5), B.EINVAL), (dict(dtype=7), B.EINVAL), (dict(D=96), B.EUNSUPPORTED),
+    (dict(D=256), B.EUNSUPPORTED), (dict(q=0), B.EINVAL), (dict(lse=0), B.EINVAL),
+    (dict(k=FAKE + 8), B.EALIGN), (dict(out=FAKE + 2), B.EALIGN), (dict(ws=0), B.EWORKSPACE),
+    (dict(wsb=16), B.EWORKSPACE),
+])
+def test_fwd_rejects_bad_arguments(lib, bad, code):
+    assert fwd(**bad) == code
+
+
+def test_workspace_bytes(lib):
+    assert B.ring_attn_fwd_workspace_bytes(1, 8, 8, 16384, 128, 8, 1, 0, 1) >= 256
+    assert B.ring_attn_fwd_workspace_bytes(1, 8, 8, 16383, 128, 8, 1, 0, 1) == 0
+    assert B.ring_attn_fwd_workspace_bytes(1, 8, 3, 16384, 128, 8, 1, 0, 1) == 0
+
+
+def test_step_and_merge_reject_bad_arguments(lib):
+    assert B.ring_attn_fwd_step(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 2, 2, 64, 64, 4, 4, 0, 1, 1, 0.1, 1, 0, FAKE, 256,
+                                None) == B.EINVAL
+    assert B.ring_attn_fwd_step(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 2, 2, 64, 64, 4, 0, -1, 1, 1, 0.1, 1, 0, FAKE,
+                                256, None) == B.EINVAL
+    assert B.ring_attn_merge(FAKE, FAKE, 0, 10, 128, FAKE, FAKE, 1, None) == B.EINVAL
+    assert B.ring_attn_merge(FAKE, FAKE, 2, 10, 12, FAKE, FAKE, 1, None) == B.EINVAL
+    assert B.ring_attn_merge(FAKE, FAKE, 2, 10, 128, FAKE, FAKE, 3, None) == B.EINVAL
+    assert B.ring_attn_merge(FAKE + 4, FAKE, 2, 10, 128, FAKE, FAKE, 1, None) == B.EALIGN
+    assert B.ring_attn_debug_watchdog(0, FAKE, 256, None) == B.EINVAL
+    assert B.ring_attn_debug_watchdog(100, FAKE, 8, None) == B.EWORKSPACE
+
+
+# ------------------------------------------------------------------ schedule
+
+def visit_counts(S, P, causal, layout, tq, tk):
+    counts = np.zeros((S, S), dtype=np.int32)
+    n = B.ring_attn_debug_visit_counts(S, P, causal, layout, tq, tk, counts.ctypes.data)
+    assert n >= 0
+    return counts, n
+
+
+@pytest.mark.parametrize("S,P", [(8, 1), (8, 2), (24, 3), (24, 8), (64, 4), (96, 8), (256, 8), (512, 16)])
+@pytest.mark.parametrize("layout", [0, 1])
+@pytest.mark.parametrize("causal", [0, 1])
+@pytest.mark.parametrize("tiles", [(4, 4), (8, 2), (6, 5), (256, 128), (64, 32)])
+def test_schedule_visits_every_allowed_pair_exactly_once(lib, S, P, layout, causal, tiles):
+    counts, _ = visit_counts(S, P, causal, layout, *tiles)
+    t = np.arange(S)[:, None]
+    u = np.arange(S)[None, :]
+    # the plain rule on global token order (the oracle's causal rule)
+    allowed = u < oracle.allowed_keys(t, S, bool(causal)) if causal else np.ones((S, S), dtype=bool)
+    np.testing.assert_array_equal(counts, allowed.astype(np.int32))
+
+
+def unit_table(Bz, Hq, Hkv, S, P, causal, layout, tq=256):
+    nmax = Bz * Hq * P * ((S // P + tq - 1) // tq)
+    buf = np.zeros((nmax, 5), dtype=np.int32)
+    n = B.ring_attn_debug_decode_units(Bz, Hq, Hkv, S, P, causal, layout, tq, buf.ctypes.data, nmax)
+    assert n == nmax
+    return buf
+
+
+@pytest.mark.parametrize("cfg", [(1, 8, 8, 16384, 8, 1, 0), (1, 8, 8, 16384, 8, 1, 1), (2, 32, 8, 131072, 16, 1, 1),
+                                 (1, 2, 2, 1024, 4, 0, 0), (1, 4, 1, 4096, 4, 1, 0), (1, 8, 8, 1 << 20, 32, 1, 1)])
+def test_units_cover_each_block_once_longest_first(lib, cfg):
+    Bz, Hq, Hkv, S, P, causal, layout = cfg
+    tab = unit_table(Bz, Hq, Hkv, S, P, causal, layout)
+    keys = {tuple(r[:4]) for r in tab}
+    nblk = (S // P + 255) // 256
+    assert len(keys) == len(tab) == Bz * Hq * P * nblk
+    cost = tab[:, 4]
+    assert (np.diff(cost) <= 0).all(), "units must be launched longest first"
+
+
+def test_gqa_group_members_are_adjacent_in_launch_order(lib):
+    tab = unit_table(2, 32, 8, 131072, 16, 1, 1)
+    # consecutive runs of 4 units share (b, kv head, shard, block) and cover the 4 query heads of the group
+    for r in range(0, 256, 4):
+        grp = tab[r:r + 4]
+        assert len({(x[0], x[1] // 4, x[2], x[3]) for x in grp}) == 1
+        assert sorted(x[1] % 4 for x in grp) == [0, 1, 2, 3]
+
+
+@pytest.mark.parametrize("layout", [0, 1])
+@pytest.mark.parametrize("causal", [0, 1])
+def test_unit_walk_follows_ring_order(lib, layout, causal):
+    S, P = 4096, 8
+    tab = unit_table(1, 1, 1, S, P, causal, layout)
+    for u in range(len(tab)):
+        i = tab[u, 2]
+        pairs = np.zeros((4096, 2), dtype=np.int32)
+        n = B.ring_attn_debug_unit_walk(1, 1, 1, S, P, causal, layout, 256, 128, u, pairs.ctypes.data, 4096)
+        assert n == tab[u, 4]
+        shards = pairs[:n, 0]
+        # ring step s meets kv shard (i - s) mod P: visiting order of distinct shards
+        order = [shards[0]] + [s for a, s in zip(shards[:-1], shards[1:]) if s != a]
+        expect = [(i - s) % P for s in range(P)]
+        if causal and layout == 0:
+            expect = [j for j in expect if j <= i]
+        assert order == expect
+        assert order[0] == i
+        # inside one shard the key tiles run 0, 1, 2, ...
+        for j in set(order):
+            kbs = pairs[:n][shards == j, 1]
+            np.testing.assert_array_equal(kbs, np.arange(len(kbs)))
+
+
+def test_schedule_info_matches_closed_form_for_1m_striped(lib):
+    info = np.zeros(6, dtype=np.int64)
+    assert B.ring_attn_debug_schedule_info(1, 8, 8, 1 << 20, 128, 32, 1, 1, info.ctypes.data) == 0
+    units, total, partial, longest, first, last = info
+    nblk = 32768 // 256
+    assert units == 8 * 32 * nblk
+    # block tb (256 rows) visits key tiles 0..2tb+1 of each of the 32 shards
+    assert total == 8 * 32 * sum(32 * (2 * tb + 2) for tb in range(nblk))
+    assert longest == first == 32 * 256 and last == 32 * 2
+    # partial tiles: the last two of every shard step of every unit
+    assert partial == 8 * 32 * nblk * 32 * 2

@@ -175,7 +175,7 @@ def oracle_sample_rate(w, q, k, v, target_seconds: float, seed_offset: int = 0):
     b = 0
     h = int(torch.randint(0, w.Hq, (1,), generator=g).item())
     n_probe = 8
-    ts = sorted(torch.randperm(w.S, generator=g)[:4096].tolist())
+    ts = torch.randperm(w.S, generator=g)[:4096].tolist()
     picked, flops, elapsed = [], 0.0, 0.0
     qh = q[b:b + 1, h:h + 1].cpu()
     g_kv = h // (w.Hq // w.Hkv)
@@ -211,7 +211,7 @@ def run_reference(args, world, rank):
         print(json.dumps({"impl": "reference", "unavailable": "workload inputs are drawn on a CUDA device"}))
         return
     q, k, v = synthetic.make_inputs(w, dev)
-    per_step = max(1.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+    per_step = max(0.2, min(args.cpu_seconds, 120.0 / max(1, args.steps + args.warmup)))
     for i in range(args.warmup):
         oracle_sample_rate(w, q, k, v, per_step / 4, seed_offset=i)
     rates, rows, secs, cores = [], 0, 0.0, 1

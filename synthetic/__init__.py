@@ -101,6 +101,11 @@ WORKLOADS = {
     "c5_bf16_s1m_striped": Workload("c5_bf16_s1m_striped", "bf16", 1, 8, 8, 1048576, 128, 32, True,
                                     "striped", 4, gen_device="cuda",
                                     description="bf16 S=1048576 P=32 causal striped"),
+    # profiling stand-in: the 1M workload's shape at 1/8 the length (inputs 0.4 GB > L2,
+    # ~45 ms per launch) so an ncu capture of every section ends in a minute or two
+    "prof_bf16_s128k_striped": Workload("prof_bf16_s128k_striped", "bf16", 1, 8, 8, 131072, 128, 32, True,
+                                        "striped", 5, gen_device="cuda",
+                                        description="bf16 S=131072 P=32 causal striped (profiling case)"),
 }
 
 

@@ -43,7 +43,7 @@ extern "C" {
 #endif
 
 #define RING_ATTN_OK 0
-#define RING_ATTN_EINVAL (-1)       /* null pointer, non-positive size, S % P != 0, Hq % Hkv != 0, bad enum */
+#define RING_ATTN_EINVAL (-1)       /* null pointer, non-positive size or scale, S % P != 0, Hq % Hkv != 0, bad enum */
 #define RING_ATTN_EALIGN (-2)       /* a tensor pointer is not 16-byte aligned */
 #define RING_ATTN_EUNSUPPORTED (-3) /* D not in {64, 128}, or no sm_100 device for the tensor-core path */
 #define RING_ATTN_EWORKSPACE (-4)   /* workspace null or smaller than ring_attn_fwd_workspace_bytes() */
@@ -80,7 +80,7 @@ size_t ring_attn_fwd_workspace_bytes(int B, int Hq, int Hkv, int64_t S, int D, i
  *   out       device pointer [B,Hq,S,D] in `dtype` (bf16 rounded to nearest even)
  *   lse       device pointer [B,Hq,S] fp32
  *   S % P == 0, Hq % Hkv == 0, D in {64, 128}; causal 0|1; layout RING_ATTN_LAYOUT_*
- *   scale     score scale (the pages use 1/sqrt(D))
+ *   scale     score scale, finite and > 0 (the pages use 1/sqrt(D))
  *   workspace device scratch of >= ring_attn_fwd_workspace_bytes() bytes
  * q/k/v must not alias out/lse.
  */
@@ -166,6 +166,14 @@ int64_t ring_attn_debug_unit_walk(int B, int Hq, int Hkv, int64_t S, int P, int 
  */
 int ring_attn_debug_schedule_info(int B, int Hq, int Hkv, int64_t S, int D, int P,
                                   int causal, int layout, int64_t* info);
+
+/*
+ * Device test of the fused kernel's software 2^x (FMA-pipe polynomial used for a
+ * fraction of the softmax exponentials): y[i] = 2^x[i] for i < n, n even, device
+ * pointers, 16-byte aligned. Relative error <= 1.02e-4 for -126 <= x <= 127;
+ * x <= -127 (including -inf) gives exactly 0.
+ */
+int ring_attn_debug_exp2(const float* x, float* y, int64_t n, void* stream);
 
 /*
  * Launches one CTA that waits on an mbarrier nobody arrives on, with a watchdog

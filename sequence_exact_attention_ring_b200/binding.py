@@ -52,6 +52,7 @@ SIGNATURES = {
     "ring_attn_debug_schedule_info": (_c_int, [_c_int, _c_int, _c_int, _c_i64, _c_int, _c_int, _c_int, _c_int,
                                                _vp]),
     "ring_attn_debug_watchdog": (_c_int, [_c_int, _vp, _c_size, _vp]),
+    "ring_attn_debug_exp2": (_c_int, [_vp, _vp, _c_i64, _vp]),
 }
 
 _lib = None
@@ -147,3 +148,7 @@ def ring_attn_debug_schedule_info(B, Hq, Hkv, S, D, P, causal, layout, info_ptr)
 
 def ring_attn_debug_watchdog(timeout_us, workspace, workspace_bytes, stream) -> int:
     return load().ring_attn_debug_watchdog(timeout_us, workspace, workspace_bytes, stream)
+
+
+def ring_attn_debug_exp2(x, y, n, stream) -> int:
+    return load().ring_attn_debug_exp2(x, y, n, stream)

@@ -1,5 +1,6 @@
 // C ABI of libringattn.so: argument validation, dispatch, status word, test hooks.
 #include <cuda_runtime.h>
+#include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -127,6 +128,7 @@ int ring_attn_fwd_algo(const void* q, const void* k, const void* v, void* out, f
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
     return RING_ATTN_EALIGN;
   if (!workspace || workspace_bytes < kWorkspaceHeaderBytes || !aligned16(workspace)) return RING_ATTN_EWORKSPACE;
+  if (!(scale > 0.f) || !isfinite(scale)) return RING_ATTN_EINVAL;
   algo = resolve_algo(algo, dtype);
   if ((rc = check_algo(algo, dtype))) return rc;
   return run_fwd(q, k, v, out, lse, g, scale, dtype, algo, 0, P, -1, 0, workspace,
@@ -151,6 +153,7 @@ int ring_attn_fwd_step(const void* q, const void* k, const void* v, float* o_par
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o_part) || !aligned16(lse_part))
     return RING_ATTN_EALIGN;
   if (!workspace || workspace_bytes < kWorkspaceHeaderBytes || !aligned16(workspace)) return RING_ATTN_EWORKSPACE;
+  if (!(scale > 0.f) || !isfinite(scale)) return RING_ATTN_EINVAL;
   algo = resolve_algo(algo, dtype);
   if ((rc = check_algo(algo, dtype))) return rc;
   const int s = ring_step_of(q_shard, kv_shard, P);
@@ -275,6 +278,12 @@ int ring_attn_debug_schedule_info(int B, int Hq, int Hkv, int64_t S, int D, int 
   return RING_ATTN_OK;
 }
 
+int ring_attn_debug_exp2(const float* x, float* y, int64_t n, void* stream) {
+  if (!x || !y || n < 0 || (n & 1)) return RING_ATTN_EINVAL;
+  if (!aligned16(x) || !aligned16(y)) return RING_ATTN_EALIGN;
+  return launch_exp2_probe(x, y, n, static_cast<cudaStream_t>(stream));
+}
+
 int ring_attn_debug_watchdog(int timeout_us, void* workspace, size_t workspace_bytes, void* stream) {
   if (timeout_us <= 0 || timeout_us > 10000000) return RING_ATTN_EINVAL;
   if (!workspace || workspace_bytes < kWorkspaceHeaderBytes) return RING_ATTN_EWORKSPACE;
@@ -302,6 +311,23 @@ __global__ void watchdog_probe_kernel(int* status, uint64_t limit_ns) {
   // nobody arrives on `bar`: the bounded wait must give up and report
   (void)mbar_wait(&bar, 0, wd);
   __syncthreads();
+}
+
+__global__ void exp2_probe_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t n) {
+  for (int64_t i = 2 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x); i < n;
+       i += 2 * (int64_t)gridDim.x * blockDim.x) {
+    const uint64_t r = exp2_poly2(f2_pack(__float_as_uint(x[i]), __float_as_uint(x[i + 1])));
+    float a, b;
+    f2_unpack(r, a, b);
+    y[i] = a;
+    y[i + 1] = b;
+  }
+}
+
+int launch_exp2_probe(const float* x, float* y, int64_t n, cudaStream_t stream) {
+  if (n == 0) return RING_ATTN_OK;
+  exp2_probe_kernel<<<148, 256, 0, stream>>>(x, y, n);
+  return cudaGetLastError() == cudaSuccess ? RING_ATTN_OK : RING_ATTN_ECUDA;
 }
 
 int launch_watchdog_probe(int timeout_us, int* status, cudaStream_t stream) {

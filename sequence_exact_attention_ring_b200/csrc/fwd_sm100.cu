@@ -14,11 +14,14 @@
 // head h) that share every K/V tile. The CTA walks the unit's KV tiles in ring
 // order (step s = 0..P-1, KV shard j = (i-s) mod P, tiles 0..n_j-1 of shard j).
 //
-// Roles (320 threads):
+// Roles (384 threads = 3 warpgroups):
 //   warps 0-3  softmax for query tile 0 (one row per thread, TMEM lanes 0..127)
 //   warps 4-7  softmax for query tile 1
 //   warp 8     TMA producer: Q once, then K and V tiles into 2-stage rings
 //   warp 9     TMEM owner; lane 0 issues every tcgen05.mma and commit
+//   warps 10-11 idle (they complete the third warpgroup for the register split)
+// Registers: launched at 168 per thread; the softmax warpgroups grow to 208 and
+// the third warpgroup shrinks to 88 (2*208 + 88 = 3*168).
 // Tensor memory (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D).
 // P (bf16) overwrites the first 64 columns of its S tile and feeds the PV MMA
 // directly from TMEM.
@@ -49,10 +52,18 @@ constexpr int NQ = 2;            // query tiles per CTA
 constexpr int BQ = BM * NQ;      // query rows per unit
 constexpr int STAGES = 2;        // K and V ring depth
 constexpr int BOXW = 64;         // bf16 elements per TMA box row (128 bytes, 128B swizzle)
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
+constexpr int kLaunchRegs = 168;     // 65536 / 384 rounded down to a multiple of 8
+constexpr int kRegsSoftmax = 208;    // per thread, warpgroups 0 and 1
+constexpr int kRegsOther = 88;       // per thread, warpgroup 2
+static_assert(2 * kRegsSoftmax + kRegsOther <= 3 * kLaunchRegs, "register split exceeds the launch pool");
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// Of every 8 column pairs of a score row, this many take 2^x from the FMA-pipe
+// polynomial (exp2_poly2) and the rest from the MUFU ex2 unit, which the tensor
+// cores would otherwise wait on (both run at 16 results/clock/SM for this shape).
+constexpr int kEmuPairsPer8 = 2;
 
 template <int D>
 struct Cfg {
@@ -150,6 +161,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int bh_kv = U.b * g.Hkv + U.h / (g.Hq / g.Hkv);
   const bool striped = g.layout == kStriped;
 
+  if (warp >= 8) {
+    regs_decrease<kRegsOther>();
   if (warp == kProducerWarp) {
     if (lane == 0) {
       // ---------------------------------------------------------------- producer
@@ -269,7 +282,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(&bars[kDrain]);
       drain_wait(&bars[kDrain], 0, p.watchdog_ns);
     }
+  }
   } else {
+    regs_increase<kRegsSoftmax>();
     // -------------------------------------------------------------------- softmax
     const int q = warp / 4;
     const int wq = warp % 4;
@@ -291,19 +306,26 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c = 0; c < BN / 32; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
       tmem_wait_ld();
-      float x[BN];
-#pragma unroll
-      for (int c = 0; c < BN; ++c) x[c] = __uint_as_float(sr[c]) * p.scale_log2;
+      // mask on the raw scores (scale > 0 keeps the order): keys b >= lim are out
       const int64_t lim = key_limit(g, U.i, w.j, a);
       const int64_t kb0 = (int64_t)w.kb * BN;
       if (kb0 + BN > lim) {
 #pragma unroll
         for (int c = 0; c < BN; ++c)
-          if (kb0 + c >= lim) x[c] = NEG_INF;
+          if (kb0 + c >= lim) sr[c] = 0xff800000u;  // -inf
       }
-      float mblk = x[0];
+      // row max: 8 independent chains of three-input max, then combine
+      float mx[8];
 #pragma unroll
-      for (int c = 1; c < BN; ++c) mblk = fmaxf(mblk, x[c]);
+      for (int ch = 0; ch < 8; ++ch) {
+        const uint32_t* v = &sr[ch * 16];
+        float m8 = fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]));
+#pragma unroll
+        for (int e = 3; e < 15; e += 2) m8 = fmax3(m8, __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+        mx[ch] = fmaxf(m8, __uint_as_float(v[15]));
+      }
+      const float mraw = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+      const float mblk = mraw * p.scale_log2;
       float alpha = 1.f;
       bool resc = false;
       if (n == 0) {
@@ -326,23 +348,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_wait_st();
       }
-      const float msub = (m_ref == NEG_INF) ? 0.f : m_ref;
-      float rs0 = 0.f, rs1 = 0.f, rs2 = 0.f, rs3 = 0.f;
+      // p = 2^(s*scale*log2e - m): one packed FMA per two scores, then ex2
+      const uint64_t c2 = f2_splat(p.scale_log2);
+      const uint64_t negm = f2_splat((m_ref == NEG_INF) ? 0.f : -m_ref);
+      uint64_t acc[4] = {0, 0, 0, 0};
       uint32_t pk[BN / 2];
 #pragma unroll
-      for (int c = 0; c < BN; c += 4) {
-        const float p0 = ex2_approx(x[c] - msub);
-        const float p1 = ex2_approx(x[c + 1] - msub);
-        const float p2 = ex2_approx(x[c + 2] - msub);
-        const float p3 = ex2_approx(x[c + 3] - msub);
-        rs0 += p0;
-        rs1 += p1;
-        rs2 += p2;
-        rs3 += p3;
+      for (int c = 0; c < BN; c += 2) {
+        const uint64_t xy = f2_fma(f2_pack(sr[c], sr[c + 1]), c2, negm);
+        uint64_t pp;
+        if ((c / 2) % 8 < kEmuPairsPer8) {
+          pp = exp2_poly2(xy);
+        } else {
+          float x0, x1;
+          f2_unpack(xy, x0, x1);
+          pp = f2_pack(__float_as_uint(ex2_approx(x0)), __float_as_uint(ex2_approx(x1)));
+        }
+        acc[(c / 2) % 4] = f2_add(acc[(c / 2) % 4], pp);
+        float p0, p1;
+        f2_unpack(pp, p0, p1);
         pk[c / 2] = pack_bf16x2(p0, p1);
-        pk[c / 2 + 1] = pack_bf16x2(p2, p3);
       }
-      l += (rs0 + rs1) + (rs2 + rs3);
+      {
+        const uint64_t t = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+        float t0, t1;
+        f2_unpack(t, t0, t1);
+        l += t0 + t1;
+      }
 #pragma unroll
       for (int c = 0; c < BN / 64; ++c) tmem_st32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[c * 32]));
       tmem_wait_st();
@@ -469,13 +501,15 @@ static int launch_impl(const void* q, const void* k, const void* v, void* out, f
   p.q_shard_only = q_shard_only;
   p.partial = partial;
   p.watchdog_ns = watchdog_ns;
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(ring_fwd_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::kSmemBytes) != cudaSuccess)
-      return RING_ATTN_ECUDA;
-    attr_set = true;
-  }
+  if (cudaFuncSetAttribute(ring_fwd_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           C::kSmemBytes) != cudaSuccess)
+    return RING_ATTN_ECUDA;
+  // The register split reallocates the block's launch pool (threads x registers at
+  // launch); refuse to launch if the compiled kernel was given fewer registers than
+  // the split needs, instead of letting setmaxnreg.inc wait forever.
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, ring_fwd_sm100_kernel<D>) != cudaSuccess) return RING_ATTN_ECUDA;
+  if (fa.numRegs * kThreads < 128 * (2 * kRegsSoftmax + kRegsOther)) return RING_ATTN_EUNSUPPORTED;
   const int64_t units = num_units(g, BQ, q_shard_only);
   if (units == 0) return RING_ATTN_OK;
   ring_fwd_sm100_kernel<D><<<(unsigned)units, kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, p);

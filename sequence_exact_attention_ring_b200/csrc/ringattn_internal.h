@@ -33,5 +33,6 @@ int launch_merge(const float* o_parts, const float* lse_parts, int n_parts, int6
                  float* lse_out, int out_dtype, cudaStream_t stream);
 
 int launch_watchdog_probe(int timeout_us, int* status, cudaStream_t stream);
+int launch_exp2_probe(const float* x, float* y, int64_t n, cudaStream_t stream);
 
 }  // namespace ringattn

@@ -53,7 +53,7 @@ GOOD = dict(B=1, Hq=4, Hkv=2, S=1024, D=128, P=4, causal=1, layout=1, dtype=1)
 FAKE = 0x10000  # aligned, never dereferenced: every call below fails validation first
 
 
-def fwd(**kw):
+def fwd(scale=0.1, **kw):
     a = dict(GOOD)
     ptrs = dict(q=FAKE, k=FAKE, v=FAKE, out=FAKE, lse=FAKE, ws=FAKE, wsb=256)
     for key in list(kw):
@@ -61,7 +61,7 @@ def fwd(**kw):
             ptrs[key] = kw.pop(key)
     a.update(kw)
     return B.ring_attn_fwd(ptrs["q"], ptrs["k"], ptrs["v"], ptrs["out"], ptrs["lse"], a["B"], a["Hq"], a["Hkv"],
-                           a["S"], a["D"], a["P"], a["causal"], a["layout"], 0.1, a["dtype"], ptrs["ws"],
+                           a["S"], a["D"], a["P"], a["causal"], a["layout"], scale, a["dtype"], ptrs["ws"],
                            ptrs["wsb"], None)
 
 
@@ -71,7 +71,8 @@ def fwd(**kw):
     (dict(layout=5), B.EINVAL), (dict(dtype=7), B.EINVAL), (dict(D=96), B.EUNSUPPORTED),
     (dict(D=256), B.EUNSUPPORTED), (dict(q=0), B.EINVAL), (dict(lse=0), B.EINVAL),
     (dict(k=FAKE + 8), B.EALIGN), (dict(out=FAKE + 2), B.EALIGN), (dict(ws=0), B.EWORKSPACE),
-    (dict(wsb=16), B.EWORKSPACE),
+    (dict(wsb=16), B.EWORKSPACE), (dict(scale=0.0), B.EINVAL), (dict(scale=-1.0), B.EINVAL),
+    (dict(scale=float("inf")), B.EINVAL), (dict(scale=float("nan")), B.EINVAL),
 ])
 def test_fwd_rejects_bad_arguments(lib, bad, code):
     assert fwd(**bad) == code

@@ -58,7 +58,9 @@ extern "C" {
 
 #define RING_ATTN_ALGO_AUTO 0    /* bf16 -> tensor-core kernel, fp32 -> SIMT kernel */
 #define RING_ATTN_ALGO_SIMT 1    /* fp32-accumulating CUDA-core kernel (fp32 or bf16 inputs) */
-#define RING_ATTN_ALGO_TCGEN05 2 /* sm_100a tcgen05/TMEM/TMA kernel (bf16 inputs only) */
+#define RING_ATTN_ALGO_TCGEN05 2 /* sm_100a tcgen05/TMEM/TMA kernel (bf16 inputs only); D=128 runs on
+                                    CTA pairs (cta_group::2), D=64 on single CTAs */
+#define RING_ATTN_ALGO_TCGEN05_1SM 3 /* the single-CTA tcgen05 kernel for every D (bf16 inputs only) */
 
 /* Library version (major*10000 + minor*100 + patch). */
 int ring_attn_version(void);

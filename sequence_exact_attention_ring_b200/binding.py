@@ -27,6 +27,7 @@ DTYPE_BF16 = 1
 ALGO_AUTO = 0
 ALGO_SIMT = 1
 ALGO_TCGEN05 = 2
+ALGO_TCGEN05_1SM = 3
 
 _c_int, _c_i64, _c_size, _vp, _c_float = ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_float
 

@@ -5,7 +5,7 @@
 #include <stdlib.h>
 #include <string.h>
 
-#include "../../include/ringattn.h"
+#include "ringattn.h"
 #include "ring_schedule.h"
 #include "ringattn_internal.h"
 #include "sm100_ptx.cuh"
@@ -70,8 +70,9 @@ int resolve_algo(int algo, int dtype) {
 }
 
 int check_algo(int algo, int dtype) {
-  if (algo != RING_ATTN_ALGO_SIMT && algo != RING_ATTN_ALGO_TCGEN05) return RING_ATTN_EINVAL;
-  if (algo == RING_ATTN_ALGO_TCGEN05 && (dtype != RING_ATTN_DTYPE_BF16 || !device_is_sm100()))
+  if (algo != RING_ATTN_ALGO_SIMT && algo != RING_ATTN_ALGO_TCGEN05 && algo != RING_ATTN_ALGO_TCGEN05_1SM)
+    return RING_ATTN_EINVAL;
+  if (algo != RING_ATTN_ALGO_SIMT && (dtype != RING_ATTN_DTYPE_BF16 || !device_is_sm100()))
     return RING_ATTN_EUNSUPPORTED;
   return RING_ATTN_OK;
 }
@@ -86,7 +87,10 @@ int run_fwd(const void* q, const void* k, const void* v, void* out, float* lse, 
             cudaStream_t stream) {
   int rc = reset_status(workspace, stream);
   if (rc) return rc;
-  if (algo == RING_ATTN_ALGO_TCGEN05)
+  if (algo == RING_ATTN_ALGO_TCGEN05 && g.D == 128)
+    return launch_fwd_sm100_2sm(q, k, v, out, lse, g, scale, s_begin, s_end, q_shard_only, partial,
+                                static_cast<int*>(workspace), watchdog_ns(), stream);
+  if (algo == RING_ATTN_ALGO_TCGEN05 || algo == RING_ATTN_ALGO_TCGEN05_1SM)
     return launch_fwd_sm100(q, k, v, out, lse, g, scale, s_begin, s_end, q_shard_only, partial,
                             static_cast<int*>(workspace), watchdog_ns(), stream);
   return launch_fwd_simt(q, k, v, out, lse, g, scale, dtype, s_begin, s_end, q_shard_only, partial, stream);

@@ -5,7 +5,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/ringattn.h"
+#include "ringattn.h"
 #include "ring_schedule.h"
 
 namespace ringattn {
@@ -13,6 +13,9 @@ namespace ringattn {
 typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                     const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                     CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// TMA map of a sharded [B, H, S, D] bf16 tensor (box: 64 elements x box_rows tokens).
+int encode_shard_map(CUtensorMap* map, const void* base, const RingGeom& g, int heads, int D, int box_rows);
 
 // Status word layout at the start of the caller's workspace.
 constexpr size_t kWorkspaceHeaderBytes = 256;
@@ -23,6 +26,12 @@ int launch_fwd_sm100(const void* q, const void* k, const void* v, void* out, flo
                      float scale, int s_begin, int s_end, int q_shard_only, int partial, int* status,
                      uint64_t watchdog_ns, cudaStream_t stream);
 int64_t fwd_sm100_units(const RingGeom& g, int q_shard_only);
+
+// The same computation on CTA pairs (cta_group::2 MMAs, D = 128 only): each CTA of
+// a pair stages half of every K and V tile.
+int launch_fwd_sm100_2sm(const void* q, const void* k, const void* v, void* out, float* lse, const RingGeom& g,
+                         float scale, int s_begin, int s_end, int q_shard_only, int partial, int* status,
+                         uint64_t watchdog_ns, cudaStream_t stream);
 
 // fp32-accumulating SIMT kernel (fp32 or bf16 inputs), same schedule and output modes.
 int launch_fwd_simt(const void* q, const void* k, const void* v, void* out, float* lse, const RingGeom& g,

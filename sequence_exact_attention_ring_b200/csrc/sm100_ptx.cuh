@@ -58,14 +58,33 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
+// How a waiting thread polls an mbarrier: 0 = try_wait (the hardware may suspend
+// the thread for a system-defined time), 1 = test_wait (never suspends),
+// 2 = try_wait with an explicit suspend-time hint of RING_ATTN_WAIT_HINT_NS.
+#ifndef RING_ATTN_WAIT_MODE
+#define RING_ATTN_WAIT_MODE 0
+#endif
+#ifndef RING_ATTN_WAIT_HINT_NS
+#define RING_ATTN_WAIT_HINT_NS 100
+#endif
+#if RING_ATTN_WAIT_MODE == 1
+#define RA_MBAR_POLL(sem) "mbarrier.test_wait.parity" sem ".shared::cta.b64 p, [%1], %2;\n\t"
+#define RA_MBAR_HINT
+#elif RING_ATTN_WAIT_MODE == 2
+#define RA_MBAR_POLL(sem) "mbarrier.try_wait.parity" sem ".shared::cta.b64 p, [%1], %2, %3;\n\t"
+#define RA_MBAR_HINT , "n"(RING_ATTN_WAIT_HINT_NS)
+#else
+#define RA_MBAR_POLL(sem) "mbarrier.try_wait.parity" sem ".shared::cta.b64 p, [%1], %2;\n\t"
+#define RA_MBAR_HINT
+#endif
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "{\n\t.reg .pred p;\n\t" RA_MBAR_POLL("")
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity) RA_MBAR_HINT
       : "memory");
   return ok != 0;
 }
@@ -87,6 +106,77 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   }
 }
 
+// ------------------------------------------------------------------ clusters (CTA pairs)
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Address of the same shared-memory location in CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Memory-ordering qualifiers of the pair barriers that other CTAs signal:
+// 0 = release/acquire at cluster scope, 1 = the instructions' defaults (CTA
+// scope), 2 = relaxed cluster-scope arrive with a CTA-scope acquire. The default
+// is 1: the data handed over is tensor memory, ordered by tcgen05.fence
+// before/after_thread_sync around the barrier, the same pairing used for
+// consumer releases of 2-SM MMA pipelines; the cluster-scope release/acquire
+// pair costs about 0.9 us per hand-over on B200.
+#ifndef RING_ATTN_CLUSTER_SEM
+#define RING_ATTN_CLUSTER_SEM 1
+#endif
+#if RING_ATTN_CLUSTER_SEM == 1
+#define RA_ARRIVE_SEM ""
+#define RA_WAIT_SEM ""
+#elif RING_ATTN_CLUSTER_SEM == 2
+#define RA_ARRIVE_SEM ".relaxed.cluster"
+#define RA_WAIT_SEM ""
+#else
+#define RA_ARRIVE_SEM ".release.cluster"
+#define RA_WAIT_SEM ".acquire.cluster"
+#endif
+
+// Arrive on an mbarrier that may live in another CTA of the cluster.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive" RA_ARRIVE_SEM ".shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t" RA_MBAR_POLL(RA_WAIT_SEM)
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity) RA_MBAR_HINT
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait with cluster-scope acquire (for barriers other CTAs of the pair signal).
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, const Watchdog& wd) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int r = 0; r < 32; ++r)
+      if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (watchdog_aborted(wd)) return false;
+    if (global_timer_ns() - t0 > wd.limit_ns) {
+      watchdog_trip(wd);
+      return false;
+    }
+  }
+}
+
 // ------------------------------------------------------------------ TMA
 // 4-D tiled bulk tensor load global -> shared, completion counted in bytes on `bar`.
 // Plain (non-multicast) form only.
@@ -96,6 +186,25 @@ __device__ __forceinline__ void tma_load_4d(void* smem_dst, const void* tmap, ui
       "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(smem_dst)),
       "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Prefetch a 4-D tile into L2 only (no shared memory, no completion signal).
+__device__ __forceinline__ void tma_prefetch_l2_4d(const void* tmap, int c0, int c1, int c2, int c3) {
+  asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
+                   reinterpret_cast<uint64_t>(tmap)),
+               "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+               : "memory");
+}
+
+// 2-SM form: data lands in this CTA's shared memory, completion bytes are counted
+// on the mbarrier at `bar_cluster_addr` (the pair leader's barrier). No multicast.
+__device__ __forceinline__ void tma_load_4d_2sm(void* smem_dst, const void* tmap, uint32_t bar_cluster_addr, int c0,
+                                                int c1, int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar_cluster_addr)
       : "memory");
 }
 
@@ -116,6 +225,47 @@ __device__ __forceinline__ void tmem_relinquish() {
 
 __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc_2sm(uint32_t* slot_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_2sm() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_2sm(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// Pair MMAs (issued by the leader CTA; operands at the same addresses in both CTAs).
+__device__ __forceinline__ void mma_ss_2sm(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ts_2sm(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive once on the barrier at this offset in every CTA of `cta_mask` when all
+// pair MMAs issued so far by this thread have completed.
+__device__ __forceinline__ void mma_commit_2sm(uint64_t* bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(cta_mask)
+      : "memory");
 }
 
 __device__ __forceinline__ void tc_fence_before() {

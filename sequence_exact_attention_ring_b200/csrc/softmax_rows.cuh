@@ -1,0 +1,137 @@
+// Row-wise pieces of the online softmax shared by the fused kernels. Each
+// softmax thread owns one query row; its scores for a block of keys sit in
+// registers as raw fp32 bits loaded from tensor memory.
+//
+// The update follows the RingAttention deep-architecture article (techknowgenie),
+// section 3: m_new = max(m_old, rowmax S), alpha = exp(m_old - m_new),
+// P = exp(S - m_new), l = l*alpha + rowsum P, O = O*alpha + P V, in base 2 with
+// scale*log2(e) folded in, and with the reference maximum moved only when the
+// block maximum exceeds it by more than kRescaleLog2 (so exponents stay <= 2^8).
+#pragma once
+
+#include <math.h>
+#include <stdint.h>
+
+#include "sm100_ptx.cuh"
+
+namespace ringattn {
+
+constexpr float kRescaleLog2 = 8.0f;
+
+// Masks keys at index >= lim (block-local: key c of the block is key kb0 + c) to -inf.
+template <int N>
+__device__ __forceinline__ void mask_scores(uint32_t (&sr)[N], int64_t kb0, int64_t lim) {
+  if (kb0 + N > lim) {
+#pragma unroll
+    for (int c = 0; c < N; ++c)
+      if (kb0 + c >= lim) sr[c] = 0xff800000u;  // -inf
+  }
+}
+
+// Maximum of N raw scores (N a multiple of 16): independent chains of three-input max.
+template <int N>
+__device__ __forceinline__ float raw_rowmax(const uint32_t (&sr)[N]) {
+  constexpr int kChains = N / 16;
+  float mx[kChains];
+#pragma unroll
+  for (int ch = 0; ch < kChains; ++ch) {
+    const uint32_t* v = &sr[ch * 16];
+    float m = fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]));
+#pragma unroll
+    for (int e = 3; e < 15; e += 2) m = fmax3(m, __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+    mx[ch] = fmaxf(m, __uint_as_float(v[15]));
+  }
+  float r = mx[0];
+#pragma unroll
+  for (int ch = 1; ch + 1 < kChains; ch += 2) r = fmax3(r, mx[ch], mx[ch + 1]);
+  if (kChains % 2 == 0) r = fmaxf(r, mx[kChains - 1]);
+  return r;
+}
+
+// p = 2^(s*scale_log2 - m) for N raw scores; packs P to bf16 pairs and returns
+// the fp32 row sum. Of every 8 column pairs, kEmu take 2^x from the FMA-pipe
+// polynomial and the rest from MUFU ex2.
+template <int N, int kEmu>
+__device__ __forceinline__ float exp_pack(const uint32_t (&sr)[N], float scale_log2, float m_sub,
+                                          uint32_t (&pk)[N / 2]) {
+  const uint64_t c2 = f2_splat(scale_log2);
+  const uint64_t negm = f2_splat(-m_sub);
+  uint64_t acc[4] = {0, 0, 0, 0};
+#pragma unroll
+  for (int c = 0; c < N; c += 2) {
+    const uint64_t xy = f2_fma(f2_pack(sr[c], sr[c + 1]), c2, negm);
+    uint64_t pp;
+    if ((c / 2) % 8 < kEmu) {
+      pp = exp2_poly2(xy);
+    } else {
+      float x0, x1;
+      f2_unpack(xy, x0, x1);
+      pp = f2_pack(__float_as_uint(ex2_approx(x0)), __float_as_uint(ex2_approx(x1)));
+    }
+    acc[(c / 2) % 4] = f2_add(acc[(c / 2) % 4], pp);
+    float p0, p1;
+    f2_unpack(pp, p0, p1);
+    pk[c / 2] = pack_bf16x2(p0, p1);
+  }
+  const uint64_t t = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+  float t0, t1;
+  f2_unpack(t, t0, t1);
+  return t0 + t1;
+}
+
+// Multiplies this warp's D accumulator columns (its 32 rows) in tensor memory by
+// each lane's alpha (1 for rows that keep their reference maximum).
+template <int D>
+__device__ __forceinline__ void rescale_o(uint32_t tO, float alpha) {
+#pragma unroll 1
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t o[32];
+    tmem_ld32(tO + c * 32, o);
+    tmem_wait_ld();
+#pragma unroll
+    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+    tmem_st32(tO + c * 32, o);
+  }
+  tmem_wait_st();
+}
+
+// Final O / l of one row: bf16 (natural token order) or fp32 partial (shard order).
+// All lanes execute the tensor-memory loads; only rows that exist are stored.
+template <int D>
+__device__ __forceinline__ void store_row(uint32_t tO, bool have_acc, bool row_ok, float inv_l, bool partial,
+                                          void* out, int64_t out_row) {
+#pragma unroll 1
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t o[32];
+    if (have_acc) {
+      tmem_ld32(tO + c * 32, o);
+      tmem_wait_ld();
+    }
+    if (!row_ok) continue;
+    if (partial) {
+      float* dst = reinterpret_cast<float*>(out) + out_row * D + c * 32;
+#pragma unroll
+      for (int e = 0; e < 32; e += 4) {
+        float4 v4;
+        v4.x = have_acc ? __uint_as_float(o[e]) * inv_l : 0.f;
+        v4.y = have_acc ? __uint_as_float(o[e + 1]) * inv_l : 0.f;
+        v4.z = have_acc ? __uint_as_float(o[e + 2]) * inv_l : 0.f;
+        v4.w = have_acc ? __uint_as_float(o[e + 3]) * inv_l : 0.f;
+        *reinterpret_cast<float4*>(dst + e) = v4;
+      }
+    } else {
+      uint32_t* dst = reinterpret_cast<uint32_t*>(reinterpret_cast<uint16_t*>(out) + out_row * D + c * 32);
+#pragma unroll
+      for (int e = 0; e < 32; e += 8) {
+        uint4 v4;
+        v4.x = pack_bf16x2(__uint_as_float(o[e]) * inv_l, __uint_as_float(o[e + 1]) * inv_l);
+        v4.y = pack_bf16x2(__uint_as_float(o[e + 2]) * inv_l, __uint_as_float(o[e + 3]) * inv_l);
+        v4.z = pack_bf16x2(__uint_as_float(o[e + 4]) * inv_l, __uint_as_float(o[e + 5]) * inv_l);
+        v4.w = pack_bf16x2(__uint_as_float(o[e + 6]) * inv_l, __uint_as_float(o[e + 7]) * inv_l);
+        *reinterpret_cast<uint4*>(dst + e / 2) = v4;
+      }
+    }
+  }
+}
+
+}  // namespace ringattn

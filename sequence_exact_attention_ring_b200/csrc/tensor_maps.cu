@@ -1,0 +1,52 @@
+// Host-side TMA tensor maps over sharded [B, H, S, D] bf16 tensors.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ring_schedule.h"
+#include "ringattn_internal.h"
+
+namespace ringattn {
+
+static PFN_encodeTiled get_encode_fn() {
+  static PFN_encodeTiled fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult qres;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qres) == cudaSuccess &&
+        qres == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_encodeTiled>(ptr);
+  }
+  return fn;
+}
+
+// 4-D view (D, local, shard, batch*heads) of a [B, H, S, D] bf16 tensor whose
+// sequence axis is split into P shards: contiguous shards are consecutive token
+// ranges, striped shards interleave with stride P. Dimensions are listed
+// innermost first so the strides grow: the striped map lists the shard before the
+// local index and kernels swap those two coordinates for it. Box: 64 elements
+// (128 bytes, 128-byte swizzle) by `box_rows` tokens of one shard.
+int encode_shard_map(CUtensorMap* map, const void* base, const RingGeom& g, int heads, int D, int box_rows) {
+  PFN_encodeTiled enc = get_encode_fn();
+  if (!enc) return RING_ATTN_ECUDA;
+  cuuint64_t dims[4];
+  cuuint64_t strides[3];
+  cuuint32_t box[4];
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const uint64_t row = (uint64_t)D * 2;
+  if (g.layout == kStriped) {
+    dims[0] = D; dims[1] = g.P; dims[2] = g.Sq; dims[3] = (uint64_t)g.B * heads;
+    strides[0] = row; strides[1] = row * g.P; strides[2] = row * g.S;
+    box[0] = 64; box[1] = 1; box[2] = box_rows; box[3] = 1;
+  } else {
+    dims[0] = D; dims[1] = g.Sq; dims[2] = g.P; dims[3] = (uint64_t)g.B * heads;
+    strides[0] = row; strides[1] = row * g.Sq; strides[2] = row * g.S;
+    box[0] = 64; box[1] = box_rows; box[2] = 1; box[3] = 1;
+  }
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? RING_ATTN_OK : RING_ATTN_ECUDA;
+}
+
+}  // namespace ringattn

@@ -28,6 +28,10 @@ SMALL = [
     (1, 2, 2, 2048, 128, 1, True, "contiguous", "bf16", "tcgen05"),  # P=1: plain causal attention
     (1, 2, 2, 96, 128, 96, True, "striped", "bf16", "tcgen05"),      # P=S: one token per shard
     (1, 2, 2, 1000, 128, 8, False, "striped", "bf16", "tcgen05"),    # non-causal, Sq=125
+    (1, 2, 2, 800, 128, 4, True, "striped", "bf16", "tcgen05_1sm"),
+    (2, 4, 2, 1536, 128, 3, True, "contiguous", "bf16", "tcgen05_1sm"),
+    (1, 2, 2, 1000, 128, 8, False, "striped", "bf16", "tcgen05_1sm"),
+    (1, 2, 2, 1100, 128, 1, True, "contiguous", "bf16", "tcgen05"),    # ragged tail inside a 512-row pair block
     (1, 3, 3, 640, 128, 2, True, "striped", "bf16", "simt"),
     (1, 2, 2, 384, 64, 4, False, "contiguous", "bf16", "simt"),
 ]
@@ -72,7 +76,7 @@ def test_layouts_and_kernels_agree(cuda_lib):
     base = (1, 4, 2, 2048, 128, 8, True)
     res = {}
     for layout in ("contiguous", "striped"):
-        for algo in ("tcgen05", "simt"):
+        for algo in ("tcgen05", "tcgen05_1sm", "simt"):
             _, _, _, _, out, lse = run_case(*base, layout, "bf16", algo, seed=77)
             res[(layout, algo)] = (out.float(), lse)
     ref_o, ref_l = res[("contiguous", "simt")]

@@ -11,7 +11,8 @@ from sequence_exact_attention_ring_b200 import binding, merge, ring_attention, r
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("algo,dtype", [("tcgen05", "bf16"), ("simt", "bf16"), ("simt", "fp32")])
+@pytest.mark.parametrize("algo,dtype", [("tcgen05", "bf16"), ("tcgen05_1sm", "bf16"), ("simt", "bf16"),
+                                        ("simt", "fp32")])
 @pytest.mark.parametrize("layout", ["contiguous", "striped"])
 def test_ring_steps_merged_equal_full_forward(cuda_lib, algo, dtype, layout):
     """Device i's P ring steps (one literal block each), merged, give the fused result."""

@@ -67,6 +67,10 @@ constexpr int kRegsSoftmax = 208;    // per thread, warpgroups 0 and 1
 constexpr int kRegsOther = 88;       // per thread, warpgroup 2
 static_assert(2 * kRegsSoftmax + kRegsOther <= 3 * kLaunchRegs, "register split exceeds the launch pool");
 constexpr int kProducerWarp = 8;
+#ifndef RING_ATTN_PRODUCER_SLEEP_NS
+#define RING_ATTN_PRODUCER_SLEEP_NS 64
+#endif
+constexpr uint32_t kProducerSleepNs = RING_ATTN_PRODUCER_SLEEP_NS;  // the producer polls slots this often
 constexpr int kMmaWarp = 9;
 // Of every 8 column pairs of a score row, this many take 2^x from the FMA-pipe
 // polynomial (exp2_poly2) and the rest from the MUFU ex2 unit, which the tensor
@@ -218,7 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kv = 0; kv < 2 && ok; ++kv, ++n) {
           const int slot = n % C::kSlots;
           const uint32_t ph = (uint32_t)(n / C::kSlots) & 1;
-          if (!(ok = mbar_wait(&empty[slot], ph ^ 1, wd))) break;
+          if (!(ok = mbar_wait_backoff<false>(&empty[slot], ph ^ 1, wd, kProducerSleepNs))) break;
           mbar_arrive_expect_tx(&full[slot], C::kTileBytes);
           const void* tm = kv == 0 ? static_cast<const void*>(&tm_k) : static_cast<const void*>(&tm_v);
           for (int bx = 0; bx < C::kBoxes; ++bx) {
@@ -334,8 +338,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < BN / 32; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
       tmem_wait_ld();
       // mask on the raw scores (scale > 0 keeps the order): keys b >= lim are out
-      mask_scores<BN>(sr, (int64_t)w.kb * BN, key_limit(g, U.i, w.j, a));
-      const float mblk = raw_rowmax<BN>(sr) * p.scale_log2;
+      const int cut = visible_keys<BN>((int64_t)w.kb * BN, key_limit(g, U.i, w.j, a));
+      mask_scores<BN>(sr, cut);
+      // a block no row of this warp can see contributes nothing: P = 0, state unchanged
+      const bool warp_empty = __all_sync(0xffffffffu, cut == 0);
+      const float mblk = warp_empty ? -INFINITY : raw_rowmax<BN>(sr) * p.scale_log2;
       float alpha = 1.f;
       bool resc = false;
       if (n == 0) {
@@ -349,7 +356,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       // S ready for tile n implies PV(n-1) of this query tile completed: O is stable
       if (__any_sync(0xffffffffu, resc)) rescale_o<D>(tO, alpha);
       uint32_t pk[BN / 2];
-      l += exp_pack<BN, kEmuPairsPer8>(sr, p.scale_log2, (m_ref == NEG_INF) ? 0.f : m_ref, pk);
+      if (warp_empty) {
+#pragma unroll
+        for (int c = 0; c < BN / 2; ++c) pk[c] = 0u;
+      } else {
+        l += exp_pack<BN, kEmuPairsPer8>(sr, p.scale_log2, (m_ref == NEG_INF) ? 0.f : m_ref, pk);
+      }
 #pragma unroll
       for (int c = 0; c < BN / 64; ++c) tmem_st32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[c * 32]));
       tmem_wait_st();

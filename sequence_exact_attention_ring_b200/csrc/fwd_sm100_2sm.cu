@@ -45,11 +45,22 @@ constexpr int kRegsSoftmax = 208;
 constexpr int kRegsOther = 88;
 static_assert(2 * kRegsSoftmax + kRegsOther <= 3 * kLaunchRegs, "register split exceeds the launch pool");
 constexpr int kProducerWarp = 8;
+#ifndef RING_ATTN_PRODUCER_SLEEP_NS
+#define RING_ATTN_PRODUCER_SLEEP_NS 64
+#endif
+constexpr uint32_t kProducerSleepNs = RING_ATTN_PRODUCER_SLEEP_NS;  // the producer polls slots this often
 constexpr int kMmaWarp = 9;
 #ifndef RING_ATTN_EMU_PAIRS_PER8
 #define RING_ATTN_EMU_PAIRS_PER8 0
 #endif
 constexpr int kEmuPairsPer8 = RING_ATTN_EMU_PAIRS_PER8;
+#ifndef RING_ATTN_MMA_SPIN
+#define RING_ATTN_MMA_SPIN 0
+#endif
+// The MMA issuer's P-ready waits: 1 = poll without suspending.
+__device__ __forceinline__ bool wait_p_ready(uint64_t* bar, uint32_t parity, const Watchdog& wd) {
+  return RING_ATTN_MMA_SPIN ? mbar_wait_spin(bar, parity, wd) : mbar_wait_cluster(bar, parity, wd);
+}
 constexpr uint16_t kPairMask = 0x3;
 
 constexpr int kSmemLimit = 232448;
@@ -171,7 +182,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int kv = 0; kv < 2; ++kv, ++n) {
           const int slot = n % kSlots;
           const uint32_t ph = (uint32_t)(n / kSlots) & 1;
-          if (!(ok = mbar_wait_cluster(&empty[slot], ph ^ 1, wd))) break;
+          if (!(ok = mbar_wait_backoff<true>(&empty[slot], ph ^ 1, wd, kProducerSleepNs))) break;
           if (leader) mbar_arrive_expect_tx(&full[slot], kCtas * kHalfBytes);
           const uint32_t leader_full = mapa_shared(smem_u32(&full[slot]), 0);
           uint8_t* dst = smem + kOffKV + slot * kHalfBytes;
@@ -246,7 +257,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (int64_t n = 0; ok && n < N; ++n) {
         const bool more = n + 1 < N;
         if (!(ok = mbar_wait_cluster(&full[vslot(n)], vphase(n), wd))) break;
-        if (!(ok = mbar_wait_cluster(&bars[kPReady + 0], (uint32_t)(n & 1), wd))) break;
+        if (!(ok = wait_p_ready(&bars[kPReady + 0], (uint32_t)(n & 1), wd))) break;
         tc_fence_after();
         issue_pv(0, vslot(n), n == 0);
         if (more) {
@@ -257,7 +268,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         } else {
           mma_commit_2sm(&bars[kODone + 0], kPairMask);
         }
-        if (!(ok = mbar_wait_cluster(&bars[kPReady + 1], (uint32_t)(n & 1), wd))) break;
+        if (!(ok = wait_p_ready(&bars[kPReady + 1], (uint32_t)(n & 1), wd))) break;
         tc_fence_after();
         issue_pv(1, vslot(n), n == 0);
         mma_commit_2sm(&empty[vslot(n)], kPairMask);
@@ -299,8 +310,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c = 0; c < BN / 32; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
       tmem_wait_ld();
-      mask_scores<BN>(sr, (int64_t)w.kb * BN, key_limit(g, U.i, w.j, a));
-      const float mblk = raw_rowmax<BN>(sr) * p.scale_log2;
+      const int cut = visible_keys<BN>((int64_t)w.kb * BN, key_limit(g, U.i, w.j, a));
+      mask_scores<BN>(sr, cut);
+      // a block no row of this warp can see contributes nothing: P = 0, state unchanged
+      const bool warp_empty = __all_sync(0xffffffffu, cut == 0);
+      const float mblk = warp_empty ? -INFINITY : raw_rowmax<BN>(sr) * p.scale_log2;
       float alpha = 1.f;
       bool resc = false;
       if (n == 0) {
@@ -314,7 +328,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // S ready for tile n implies PV(n-1) of this query tile completed: O is stable
       if (__any_sync(0xffffffffu, resc)) rescale_o<D>(tO, alpha);
       uint32_t pk[BN / 2];
-      l += exp_pack<BN, kEmuPairsPer8>(sr, p.scale_log2, (m_ref == NEG_INF) ? 0.f : m_ref, pk);
+      if (warp_empty) {
+#pragma unroll
+        for (int c = 0; c < BN / 2; ++c) pk[c] = 0u;
+      } else {
+        l += exp_pack<BN, kEmuPairsPer8>(sr, p.scale_log2, (m_ref == NEG_INF) ? 0.f : m_ref, pk);
+      }
 #pragma unroll
       for (int c = 0; c < BN / 64; ++c) tmem_st32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[c * 32]));
       tmem_wait_st();

@@ -161,6 +161,56 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
   return ok != 0;
 }
 
+// Bounded wait that sleeps `sleep_ns` between polls: for waiters off the critical
+// path (a producer running ahead), so their polling does not take issue slots
+// from the warps doing the math on the same scheduler.
+template <bool kCluster>
+__device__ __forceinline__ bool mbar_wait_backoff(uint64_t* bar, uint32_t parity, const Watchdog& wd,
+                                                  uint32_t sleep_ns) {
+  auto poll = [&]() { return kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
+  if (poll()) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    __nanosleep(sleep_ns);
+    if (poll()) return true;
+    if (watchdog_aborted(wd)) return false;
+    if (global_timer_ns() - t0 > wd.limit_ns) {
+      watchdog_trip(wd);
+      return false;
+    }
+  }
+}
+
+// Bounded wait that never suspends the thread (mbarrier.test_wait): for a single
+// thread on the critical path whose wake-up latency matters more than the issue
+// slots its polling takes from other warps.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, const Watchdog& wd) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int r = 0; r < 64; ++r)
+      if (mbar_test_wait(bar, parity)) return true;
+    if (watchdog_aborted(wd)) return false;
+    if (global_timer_ns() - t0 > wd.limit_ns) {
+      watchdog_trip(wd);
+      return false;
+    }
+  }
+}
+
 // Bounded wait with cluster-scope acquire (for barriers other CTAs of the pair signal).
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, const Watchdog& wd) {
   if (mbar_try_wait_cluster(bar, parity)) return true;

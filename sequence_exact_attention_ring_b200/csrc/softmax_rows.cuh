@@ -18,13 +18,19 @@ namespace ringattn {
 
 constexpr float kRescaleLog2 = 8.0f;
 
-// Masks keys at index >= lim (block-local: key c of the block is key kb0 + c) to -inf.
+// Number of keys of the block starting at key kb0 that are visible (keys < lim), in [0, N].
 template <int N>
-__device__ __forceinline__ void mask_scores(uint32_t (&sr)[N], int64_t kb0, int64_t lim) {
-  if (kb0 + N > lim) {
+__device__ __forceinline__ int visible_keys(int64_t kb0, int64_t lim) {
+  const int64_t v = lim - kb0;
+  return v <= 0 ? 0 : (v >= N ? N : (int)v);
+}
+
+// Masks block-local keys c >= cut to -inf (a no-op when cut == N).
+template <int N>
+__device__ __forceinline__ void mask_scores(uint32_t (&sr)[N], int cut) {
+  if (cut < N) {
 #pragma unroll
-    for (int c = 0; c < N; ++c)
-      if (kb0 + c >= lim) sr[c] = 0xff800000u;  // -inf
+    for (int c = 0; c < N; ++c) sr[c] = c < cut ? sr[c] : 0xff800000u;  // -inf
   }
 }
 

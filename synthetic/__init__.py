@@ -106,6 +106,10 @@ WORKLOADS = {
     "prof_bf16_s128k_striped": Workload("prof_bf16_s128k_striped", "bf16", 1, 8, 8, 131072, 128, 32, True,
                                         "striped", 5, gen_device="cuda",
                                         description="bf16 S=131072 P=32 causal striped (profiling case)"),
+    # twice the length: with the 128k case it shows whether DRAM traffic grows with the work
+    "prof_bf16_s256k_striped": Workload("prof_bf16_s256k_striped", "bf16", 1, 8, 8, 262144, 128, 32, True,
+                                        "striped", 6, gen_device="cuda",
+                                        description="bf16 S=262144 P=32 causal striped (profiling case)"),
 }
 
 

@@ -131,6 +131,37 @@ int ring_attn_merge(const float* o_parts, const float* lse_parts, int n_parts, i
  */
 int ring_attn_status(const void* workspace, void* stream);
 
+/*
+ * ring_attn_fwd without a caller workspace. The method described by the pages has no
+ * counterpart; this is a library convenience. It is for callers that cannot allocate
+ * device memory: a plain C/C++ host that links only this library and has no device
+ * allocator of its own, or a process whose device memory is planned up front and
+ * which treats any later allocation as an error.
+ *
+ * The scratch (status word included) is a static __device__ array of this library,
+ * RING_ATTN_NOALLOC_SCRATCH_BYTES bytes per device. Neither the call nor its one-time
+ * setup calls cudaMalloc, cudaFree or any other allocating routine.
+ *   Arguments q ... dtype, stream: as ring_attn_fwd.
+ *   scratch_out  optional host pointer (may be NULL). On success it receives the
+ *                device address of this device's scratch. Pass that address to
+ *                ring_attn_status() to read the status word of the last call.
+ * Setup: the first call on each device, with that device current, looks up the
+ * array's device address (cudaGetSymbolAddress) and caches it. Make that first
+ * call before any stream capture on that device.
+ * Errors: as ring_attn_fwd. If these arguments need more workspace than the array
+ * holds, it returns RING_ATTN_EWORKSPACE and enqueues nothing. If the address
+ * lookup fails, it returns RING_ATTN_ECUDA.
+ * Concurrency: every call on a device shares one scratch array. Calls that overlap
+ * on the device (different streams, or host threads without ordering) race on the
+ * status word. Order them on one stream, or use ring_attn_fwd with separate
+ * workspaces.
+ */
+#define RING_ATTN_NOALLOC_SCRATCH_BYTES 4096
+int ring_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* out, float* lse,
+                          int B, int Hq, int Hkv, int64_t S, int D, int P,
+                          int causal, int layout, float scale, int dtype,
+                          void* stream, void** scratch_out);
+
 /* ---- test hooks ------------------------------------------------------------ */
 
 /*

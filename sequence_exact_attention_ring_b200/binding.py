@@ -45,6 +45,8 @@ SIGNATURES = {
                                     _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _c_int, _vp, _c_size, _vp]),
     "ring_attn_merge": (_c_int, [_vp, _vp, _c_int, _c_i64, _c_int, _vp, _vp, _c_int, _vp]),
     "ring_attn_status": (_c_int, [_vp, _vp]),
+    "ring_attn_fwd_noalloc": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_i64, _c_int, _c_int,
+                                       _c_int, _c_int, _c_float, _c_int, _vp, ctypes.POINTER(_vp)]),
     "ring_attn_debug_visit_counts": (_c_i64, [_c_i64, _c_int, _c_int, _c_int, _c_int, _c_int, _vp]),
     "ring_attn_debug_decode_units": (_c_int, [_c_int, _c_int, _c_int, _c_i64, _c_int, _c_int, _c_int, _c_int,
                                               _vp, _c_i64]),
@@ -128,6 +130,14 @@ def ring_attn_merge(o_parts, lse_parts, n_parts, rows, D, out, lse_out, out_dtyp
 
 def ring_attn_status(workspace, stream) -> int:
     return load().ring_attn_status(workspace, stream)
+
+
+def ring_attn_fwd_noalloc(q, k, v, out, lse, B, Hq, Hkv, S, D, P, causal, layout, scale, dtype, stream):
+    """Returns (code, device address of the library's scratch for this device or None)."""
+    scratch = _vp()
+    rc = load().ring_attn_fwd_noalloc(q, k, v, out, lse, B, Hq, Hkv, S, D, P, causal, layout, scale, dtype, stream,
+                                      ctypes.byref(scratch))
+    return rc, scratch.value
 
 
 def ring_attn_debug_visit_counts(S, P, causal, layout, tile_q, tile_k, counts_ptr) -> int:

@@ -213,24 +213,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         while (global_timer_ns() - t0 < 2000000ull) {
         }
       }
-    } else if (warp == kMmaWarp && lane == 0 && leader) {
+    } else if (warp == kMmaWarp && leader) {
       // ---------------------------------------------------------------- MMA issuer (leader only)
+      // The whole warp runs this loop and waits on the barriers; one elected lane
+      // issues each tcgen05 instruction. Descriptor bases are built once; every MMA
+      // then adds a compile-time offset (address >> 4) to the start-address field.
       const int64_t N = unit_tile_count(g, U.i, a_hi, BN, p.s_begin, p.s_end);
       const uint32_t sbase = smem_u32(smem);
-      // Descriptor bases are built once; every MMA then only adds a compile-time
-      // offset (address >> 4) to the start-address field, keeping the issuing thread
-      // lean while it shares its scheduler with the softmax warps.
       const uint64_t dq0 = smem_desc_sw128(sbase + kOffQ, 0, 1024);
       const uint64_t dk0 = smem_desc_sw128(sbase + kOffKV, 0, 1024);
       const uint64_t dv0 = smem_desc_sw128(sbase + kOffKV, kHalfBytes, 1024);
+      const bool issuer = elect_one_sync();
       auto issue_s = [&](int q, int slot) {
         const uint64_t dq = dq0 + (uint64_t)((q * kQTileBytes) >> 4);
         const uint64_t dk = dk0 + (uint64_t)((slot * kHalfBytes) >> 4);
         const uint32_t d = tmem + kColS + q * BN;
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
-          mma_ss_2sm(d, dq + (((k / 4) * kQBoxBytes + (k % 4) * 32) >> 4),
-                     dk + (((k / 4) * kKBoxBytes + (k % 4) * 32) >> 4), kIdescQK, k > 0);
+          if (issuer)
+            mma_ss_2sm(d, dq + (((k / 4) * kQBoxBytes + (k % 4) * 32) >> 4),
+                       dk + (((k / 4) * kKBoxBytes + (k % 4) * 32) >> 4), kIdescQK, k > 0);
       };
       auto issue_pv = [&](int q, int slot, bool first) {
         const uint64_t dv = dv0 + (uint64_t)((slot * kHalfBytes) >> 4);
@@ -238,50 +240,55 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t pa = tmem + kColS + q * BN;
 #pragma unroll
         for (int k = 0; k < BN / 16; ++k)
-          mma_ts_2sm(d, pa + k * 8, dv + ((k * 16 * 128) >> 4), kIdescPV, !(first && k == 0));
+          if (issuer) mma_ts_2sm(d, pa + k * 8, dv + ((k * 16 * 128) >> 4), kIdescPV, !(first && k == 0));
       };
+      auto commit = [&](uint64_t* bar) {
+        if (issuer) mma_commit_2sm(bar, kPairMask);
+      };
+      // every lane polls; the warp proceeds only if all lanes saw the phase complete
+      auto wait_all = [&](bool r) { return __all_sync(0xffffffffu, r); };
       auto kslot = [&](int64_t n) { return (int)((2 * n) % kSlots); };
       auto kphase = [&](int64_t n) { return (uint32_t)(((2 * n) / kSlots) & 1); };
       auto vslot = [&](int64_t n) { return (int)((2 * n + 1) % kSlots); };
       auto vphase = [&](int64_t n) { return (uint32_t)(((2 * n + 1) / kSlots) & 1); };
-      bool ok = N > 0 && mbar_wait_cluster(&bars[kQFull], 0, wd);
-      if (ok) ok = mbar_wait_cluster(&full[kslot(0)], kphase(0), wd);
+      bool ok = N > 0 && wait_all(mbar_wait_cluster(&bars[kQFull], 0, wd));
+      if (ok) ok = wait_all(mbar_wait_cluster(&full[kslot(0)], kphase(0), wd));
       if (ok) {
         tc_fence_after();
         issue_s(0, kslot(0));
-        mma_commit_2sm(&bars[kSFull + 0], kPairMask);
+        commit(&bars[kSFull + 0]);
         issue_s(1, kslot(0));
-        mma_commit_2sm(&bars[kSFull + 1], kPairMask);
-        mma_commit_2sm(&empty[kslot(0)], kPairMask);
+        commit(&bars[kSFull + 1]);
+        commit(&empty[kslot(0)]);
       }
       for (int64_t n = 0; ok && n < N; ++n) {
         const bool more = n + 1 < N;
-        if (!(ok = mbar_wait_cluster(&full[vslot(n)], vphase(n), wd))) break;
-        if (!(ok = wait_p_ready(&bars[kPReady + 0], (uint32_t)(n & 1), wd))) break;
+        if (!(ok = wait_all(mbar_wait_cluster(&full[vslot(n)], vphase(n), wd)))) break;
+        if (!(ok = wait_all(wait_p_ready(&bars[kPReady + 0], (uint32_t)(n & 1), wd)))) break;
         tc_fence_after();
         issue_pv(0, vslot(n), n == 0);
         if (more) {
-          if (!(ok = mbar_wait_cluster(&full[kslot(n + 1)], kphase(n + 1), wd))) break;
+          if (!(ok = wait_all(mbar_wait_cluster(&full[kslot(n + 1)], kphase(n + 1), wd)))) break;
           tc_fence_after();
           issue_s(0, kslot(n + 1));
-          mma_commit_2sm(&bars[kSFull + 0], kPairMask);
+          commit(&bars[kSFull + 0]);
         } else {
-          mma_commit_2sm(&bars[kODone + 0], kPairMask);
+          commit(&bars[kODone + 0]);
         }
-        if (!(ok = wait_p_ready(&bars[kPReady + 1], (uint32_t)(n & 1), wd))) break;
+        if (!(ok = wait_all(wait_p_ready(&bars[kPReady + 1], (uint32_t)(n & 1), wd)))) break;
         tc_fence_after();
         issue_pv(1, vslot(n), n == 0);
-        mma_commit_2sm(&empty[vslot(n)], kPairMask);
+        commit(&empty[vslot(n)]);
         if (more) {
           issue_s(1, kslot(n + 1));
-          mma_commit_2sm(&bars[kSFull + 1], kPairMask);
-          mma_commit_2sm(&empty[kslot(n + 1)], kPairMask);
+          commit(&bars[kSFull + 1]);
+          commit(&empty[kslot(n + 1)]);
         } else {
-          mma_commit_2sm(&bars[kODone + 1], kPairMask);
+          commit(&bars[kODone + 1]);
         }
       }
       // both CTAs learn when every pair MMA has finished (before TMEM is released)
-      mma_commit_2sm(&bars[kDrain], kPairMask);
+      commit(&bars[kDrain]);
       drain_wait(&bars[kDrain], 0, p.watchdog_ns);
     } else if (warp == kMmaWarp && lane == 0) {
       drain_wait(&bars[kDrain], 0, p.watchdog_ns);

@@ -318,6 +318,19 @@ __device__ __forceinline__ void mma_commit_2sm(uint64_t* bar, uint16_t cta_mask)
       : "memory");
 }
 
+// True in exactly one active lane of a converged warp (elect.sync). Code that issues
+// tcgen05 instructions runs warp-wide and guards only the issuing instruction with
+// this predicate, so descriptor arithmetic stays in warp-uniform registers.
+__device__ __forceinline__ bool elect_one_sync() {
+  uint32_t e = 0;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "elect.sync _|P, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(e));
+  return e != 0;
+}
+
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }

@@ -1,6 +1,6 @@
-// Row-wise pieces of the online softmax shared by the fused kernels. Each
-// softmax thread owns one query row; its scores for a block of keys sit in
-// registers as raw fp32 bits loaded from tensor memory.
+// Row-wise pieces of the online softmax shared by the fused kernels. A softmax
+// thread owns one query row, or one half of its key columns; its scores for a
+// block of keys sit in registers as raw fp32 bits loaded from tensor memory.
 //
 // The update follows the RingAttention deep-architecture article (techknowgenie),
 // section 3: m_new = max(m_old, rowmax S), alpha = exp(m_old - m_new),
@@ -85,12 +85,12 @@ __device__ __forceinline__ float exp_pack(const uint32_t (&sr)[N], float scale_l
   return t0 + t1;
 }
 
-// Multiplies this warp's D accumulator columns (its 32 rows) in tensor memory by
+// Multiplies kCols accumulator columns of this warp's 32 rows in tensor memory by
 // each lane's alpha (1 for rows that keep their reference maximum).
-template <int D>
+template <int kCols>
 __device__ __forceinline__ void rescale_o(uint32_t tO, float alpha) {
 #pragma unroll 1
-  for (int c = 0; c < D / 32; ++c) {
+  for (int c = 0; c < kCols / 32; ++c) {
     uint32_t o[32];
     tmem_ld32(tO + c * 32, o);
     tmem_wait_ld();
@@ -101,21 +101,24 @@ __device__ __forceinline__ void rescale_o(uint32_t tO, float alpha) {
   tmem_wait_st();
 }
 
-// Final O / l of one row: bf16 (natural token order) or fp32 partial (shard order).
-// All lanes execute the tensor-memory loads; only rows that exist are stored.
-template <int D>
-__device__ __forceinline__ void store_row(uint32_t tO, bool have_acc, bool row_ok, float inv_l, bool partial,
-                                          void* out, int64_t out_row) {
+// Final O / l of kCols accumulator columns of one row, written to columns
+// [col0, col0 + kCols) of an output row of row_stride elements: bf16 (natural token
+// order) or fp32 partial (shard order). All lanes execute the tensor-memory loads;
+// only rows that exist are stored.
+template <int kCols>
+__device__ __forceinline__ void store_row_cols(uint32_t tO, bool have_acc, bool row_ok, float inv_l, bool partial,
+                                               void* out, int64_t out_row, int row_stride, int col0) {
 #pragma unroll 1
-  for (int c = 0; c < D / 32; ++c) {
+  for (int c = 0; c < kCols / 32; ++c) {
     uint32_t o[32];
     if (have_acc) {
       tmem_ld32(tO + c * 32, o);
       tmem_wait_ld();
     }
     if (!row_ok) continue;
+    const int64_t base = out_row * row_stride + col0 + c * 32;
     if (partial) {
-      float* dst = reinterpret_cast<float*>(out) + out_row * D + c * 32;
+      float* dst = reinterpret_cast<float*>(out) + base;
 #pragma unroll
       for (int e = 0; e < 32; e += 4) {
         float4 v4;
@@ -126,7 +129,7 @@ __device__ __forceinline__ void store_row(uint32_t tO, bool have_acc, bool row_o
         *reinterpret_cast<float4*>(dst + e) = v4;
       }
     } else {
-      uint32_t* dst = reinterpret_cast<uint32_t*>(reinterpret_cast<uint16_t*>(out) + out_row * D + c * 32);
+      uint32_t* dst = reinterpret_cast<uint32_t*>(reinterpret_cast<uint16_t*>(out) + base);
 #pragma unroll
       for (int e = 0; e < 32; e += 8) {
         uint4 v4;
@@ -138,6 +141,13 @@ __device__ __forceinline__ void store_row(uint32_t tO, bool have_acc, bool row_o
       }
     }
   }
+}
+
+// Final O / l of a whole row of D columns.
+template <int D>
+__device__ __forceinline__ void store_row(uint32_t tO, bool have_acc, bool row_ok, float inv_l, bool partial,
+                                          void* out, int64_t out_row) {
+  store_row_cols<D>(tO, have_acc, row_ok, inv_l, partial, out, out_row, D, 0);
 }
 
 }  // namespace ringattn

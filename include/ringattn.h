@@ -14,9 +14,12 @@
  * order of the work. Causal masking (section 7 "causal attention with striped
  * attention") lets query token t see keys u <= t (inclusive diagonal). Layout
  * CONTIGUOUS puts tokens [i*Sq, (i+1)*Sq) on shard i; STRIPED puts token t on
- * shard t mod P.
+ * shard t mod P. ZIGZAG (named as a causal load balancer by the RingAttention
+ * newsletter on cmlonder, section "claim and reality", without a definition) is
+ * read as: cut the sequence into 2P chunks of C = S/(2P) tokens and give shard i
+ * chunks i and 2P-1-i, so every shard folds the same causal work.
  *
- * Tensor layout (all row-major, contiguous, natural token order for both layouts):
+ * Tensor layout (all row-major, contiguous, natural token order for every layout):
  *     q, out : [B, Hq,  S, D]      k, v : [B, Hkv, S, D]      lse : [B, Hq, S] fp32
  * Query head h reads KV head h / (Hq/Hkv) (grouped-query attention when Hkv < Hq).
  * lse = m + ln(l): natural log-sum-exp of the scaled scores of each row.
@@ -43,7 +46,7 @@ extern "C" {
 #endif
 
 #define RING_ATTN_OK 0
-#define RING_ATTN_EINVAL (-1)       /* null pointer, non-positive size or scale, S % P != 0, Hq % Hkv != 0, bad enum */
+#define RING_ATTN_EINVAL (-1)       /* null pointer, non-positive size or scale, S % P != 0 (S % 2P != 0 for zigzag), Hq % Hkv != 0, bad enum */
 #define RING_ATTN_EALIGN (-2)       /* a tensor pointer is not 16-byte aligned */
 #define RING_ATTN_EUNSUPPORTED (-3) /* D not in {64, 128}, or no sm_100 device for the tensor-core path */
 #define RING_ATTN_EWORKSPACE (-4)   /* workspace null or smaller than ring_attn_fwd_workspace_bytes() */
@@ -52,6 +55,7 @@ extern "C" {
 
 #define RING_ATTN_LAYOUT_CONTIGUOUS 0
 #define RING_ATTN_LAYOUT_STRIPED 1
+#define RING_ATTN_LAYOUT_ZIGZAG 2 /* needs S % (2P) == 0; the tensor-core kernels also need (S/(2P)) % 128 == 0 */
 
 #define RING_ATTN_DTYPE_FP32 0
 #define RING_ATTN_DTYPE_BF16 1
@@ -82,6 +86,7 @@ size_t ring_attn_fwd_workspace_bytes(int B, int Hq, int Hkv, int64_t S, int D, i
  *   out       device pointer [B,Hq,S,D] in `dtype` (bf16 rounded to nearest even)
  *   lse       device pointer [B,Hq,S] fp32
  *   S % P == 0, Hq % Hkv == 0, D in {64, 128}; causal 0|1; layout RING_ATTN_LAYOUT_*
+ *             (AUTO runs zigzag shapes the tensor-core kernels cannot tile on the SIMT kernel)
  *   scale     score scale, finite and > 0 (the pages use 1/sqrt(D))
  *   workspace device scratch of >= ring_attn_fwd_workspace_bytes() bytes
  * q/k/v must not alias out/lse.

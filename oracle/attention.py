@@ -19,6 +19,10 @@ Sources (the RingAttention pages):
   [MASK] same article, section 7 "causal attention with striped attention": a
          decoder attends to past tokens; striped layout deals tokens round-robin,
          token t on shard t mod P.
+  [ZIG]  RingAttention newsletter (cmlonder), section "claim and reality": striped or
+         zigzag schedules counter the causal load imbalance of the ring. The page
+         names zigzag without defining it; the plainest reading taken here cuts the
+         sequence into 2P equal chunks and gives shard i chunks i and 2P-1-i.
 
 Readings where the pages are silent (each also listed in the design doc):
   * lse = m + ln(l): natural log, in units of the scaled scores.
@@ -64,7 +68,8 @@ def allowed_keys(t, S: int, causal: bool):
 def shard_tokens(S: int, P: int, layout: str, i: int) -> np.ndarray:
     """Global token ids held by shard i, in local order.
 
-    contiguous: tokens [i*S/P, (i+1)*S/P); striped: tokens a*P + i for a = 0..S/P-1.
+    contiguous: tokens [i*S/P, (i+1)*S/P); striped: tokens a*P + i for a = 0..S/P-1;
+    zigzag [ZIG]: with chunks of C = S/(2P) tokens, chunk i then chunk 2P-1-i.
     """
     if S % P != 0:
         raise ValueError("S must be a multiple of P")
@@ -74,6 +79,12 @@ def shard_tokens(S: int, P: int, layout: str, i: int) -> np.ndarray:
         return i * Sq + a
     if layout == "striped":
         return a * P + i
+    if layout == "zigzag":
+        if S % (2 * P) != 0:
+            raise ValueError("zigzag needs S to be a multiple of 2P")
+        C = S // (2 * P)
+        c = np.arange(C, dtype=np.int64)
+        return np.concatenate([i * C + c, (2 * P - 1 - i) * C + c])
     raise ValueError(f"unknown layout {layout!r}")
 
 

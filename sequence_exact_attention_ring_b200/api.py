@@ -11,7 +11,7 @@ import torch
 
 from . import binding as _b
 
-_LAYOUTS = {"contiguous": _b.LAYOUT_CONTIGUOUS, "striped": _b.LAYOUT_STRIPED}
+_LAYOUTS = {"contiguous": _b.LAYOUT_CONTIGUOUS, "striped": _b.LAYOUT_STRIPED, "zigzag": _b.LAYOUT_ZIGZAG}
 _ALGOS = {"auto": _b.ALGO_AUTO, "simt": _b.ALGO_SIMT, "tcgen05": _b.ALGO_TCGEN05,
           "tcgen05_1sm": _b.ALGO_TCGEN05_1SM}
 _DTYPES = {torch.float32: _b.DTYPE_FP32, torch.bfloat16: _b.DTYPE_BF16}

@@ -22,6 +22,7 @@ ETIMEOUT = -6
 
 LAYOUT_CONTIGUOUS = 0
 LAYOUT_STRIPED = 1
+LAYOUT_ZIGZAG = 2
 DTYPE_FP32 = 0
 DTYPE_BF16 = 1
 ALGO_AUTO = 0

@@ -22,7 +22,10 @@ int check_geom(int B, int Hq, int Hkv, int64_t S, int D, int P, int causal, int 
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || S <= 0 || D <= 0 || P <= 0) return RING_ATTN_EINVAL;
   if (S % P != 0 || Hq % Hkv != 0) return RING_ATTN_EINVAL;
   if (causal != 0 && causal != 1) return RING_ATTN_EINVAL;
-  if (layout != RING_ATTN_LAYOUT_CONTIGUOUS && layout != RING_ATTN_LAYOUT_STRIPED) return RING_ATTN_EINVAL;
+  if (layout != RING_ATTN_LAYOUT_CONTIGUOUS && layout != RING_ATTN_LAYOUT_STRIPED &&
+      layout != RING_ATTN_LAYOUT_ZIGZAG)
+    return RING_ATTN_EINVAL;
+  if (layout == RING_ATTN_LAYOUT_ZIGZAG && S % (2 * (int64_t)P) != 0) return RING_ATTN_EINVAL;
   if (dtype != RING_ATTN_DTYPE_FP32 && dtype != RING_ATTN_DTYPE_BF16) return RING_ATTN_EINVAL;
   if ((int64_t)B * Hq > (1 << 24) || S > ((int64_t)1 << 31)) return RING_ATTN_EINVAL;
   if (D != 64 && D != 128) return RING_ATTN_EUNSUPPORTED;
@@ -64,15 +67,20 @@ uint64_t watchdog_ns() {
   return ns;
 }
 
-int resolve_algo(int algo, int dtype) {
-  if (algo == RING_ATTN_ALGO_AUTO) return dtype == RING_ATTN_DTYPE_BF16 ? RING_ATTN_ALGO_TCGEN05 : RING_ATTN_ALGO_SIMT;
+// The tensor-core kernels load 128-row tiles with TMA; under zigzag a tile must not
+// cross from a shard's first chunk into its second, so chunks are whole tiles.
+bool tcgen05_layout_ok(const RingGeom& g) { return g.layout != kZigzag || (g.Sq / 2) % 128 == 0; }
+
+int resolve_algo(int algo, int dtype, const RingGeom& g) {
+  if (algo == RING_ATTN_ALGO_AUTO)
+    return dtype == RING_ATTN_DTYPE_BF16 && tcgen05_layout_ok(g) ? RING_ATTN_ALGO_TCGEN05 : RING_ATTN_ALGO_SIMT;
   return algo;
 }
 
-int check_algo(int algo, int dtype) {
+int check_algo(int algo, int dtype, const RingGeom& g) {
   if (algo != RING_ATTN_ALGO_SIMT && algo != RING_ATTN_ALGO_TCGEN05 && algo != RING_ATTN_ALGO_TCGEN05_1SM)
     return RING_ATTN_EINVAL;
-  if (algo != RING_ATTN_ALGO_SIMT && (dtype != RING_ATTN_DTYPE_BF16 || !device_is_sm100()))
+  if (algo != RING_ATTN_ALGO_SIMT && (dtype != RING_ATTN_DTYPE_BF16 || !tcgen05_layout_ok(g) || !device_is_sm100()))
     return RING_ATTN_EUNSUPPORTED;
   return RING_ATTN_OK;
 }
@@ -133,8 +141,8 @@ int ring_attn_fwd_algo(const void* q, const void* k, const void* v, void* out, f
     return RING_ATTN_EALIGN;
   if (!workspace || workspace_bytes < kWorkspaceHeaderBytes || !aligned16(workspace)) return RING_ATTN_EWORKSPACE;
   if (!(scale > 0.f) || !isfinite(scale)) return RING_ATTN_EINVAL;
-  algo = resolve_algo(algo, dtype);
-  if ((rc = check_algo(algo, dtype))) return rc;
+  algo = resolve_algo(algo, dtype, g);
+  if ((rc = check_algo(algo, dtype, g))) return rc;
   return run_fwd(q, k, v, out, lse, g, scale, dtype, algo, 0, P, -1, 0, workspace,
                  static_cast<cudaStream_t>(stream));
 }
@@ -158,8 +166,8 @@ int ring_attn_fwd_step(const void* q, const void* k, const void* v, float* o_par
     return RING_ATTN_EALIGN;
   if (!workspace || workspace_bytes < kWorkspaceHeaderBytes || !aligned16(workspace)) return RING_ATTN_EWORKSPACE;
   if (!(scale > 0.f) || !isfinite(scale)) return RING_ATTN_EINVAL;
-  algo = resolve_algo(algo, dtype);
-  if ((rc = check_algo(algo, dtype))) return rc;
+  algo = resolve_algo(algo, dtype, g);
+  if ((rc = check_algo(algo, dtype, g))) return rc;
   const int s = ring_step_of(q_shard, kv_shard, P);
   return run_fwd(q, k, v, o_part, lse_part, g, scale, dtype, algo, s, s + 1, q_shard, 1, workspace,
                  static_cast<cudaStream_t>(stream));

@@ -177,7 +177,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t a_hi = (a0 + BQ - 1 < g.Sq - 1) ? a0 + BQ - 1 : g.Sq - 1;
   const int bh_q = U.b * g.Hq + U.h;
   const int bh_kv = U.b * g.Hkv + U.h / (g.Hq / g.Hkv);
-  const bool striped = g.layout == kStriped;
   const int64_t N = unit_tile_count(g, U.i, a_hi, BN, p.s_begin, p.s_end);
 
   if (warp >= 8) {
@@ -191,13 +190,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (N > 0) {
         mbar_arrive_expect_tx(&bars[kQFull], NQ * C::kTileBytes);
         for (int q = 0; q < NQ; ++q) {
-          const int row = (int)(a0 + q * BM);
+          int c1, c2;
+          shard_map_coords(g, U.i, a0 + q * BM, c1, c2);
           for (int bx = 0; bx < C::kBoxes; ++bx) {
             uint8_t* dst = smem + C::kOffQ + q * C::kTileBytes + bx * C::kBoxBytes;
-            if (striped)
-              tma_load_4d(dst, &tm_q, &bars[kQFull], bx * BOXW, U.i, row, bh_q);
-            else
-              tma_load_4d(dst, &tm_q, &bars[kQFull], bx * BOXW, row, U.i, bh_q);
+            tma_load_4d(dst, &tm_q, &bars[kQFull], bx * BOXW, c1, c2, bh_q);
           }
         }
       }
@@ -206,19 +203,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = 0; t < kPrefetchTiles && walk_valid(wp); ++t) walk_next(g, wp, a_hi, BN);
       for (; walk_valid(w); walk_next(g, w, a_hi, BN)) {
         if (kPrefetchTiles > 0 && walk_valid(wp)) {
-          const int prow = wp.kb * BN;
+          int p1, p2;
+          shard_map_coords(g, wp.j, wp.kb * BN, p1, p2);
           for (int bx = 0; bx < C::kBoxes; ++bx) {
-            if (striped) {
-              tma_prefetch_l2_4d(&tm_k, bx * BOXW, wp.j, prow, bh_kv);
-              tma_prefetch_l2_4d(&tm_v, bx * BOXW, wp.j, prow, bh_kv);
-            } else {
-              tma_prefetch_l2_4d(&tm_k, bx * BOXW, prow, wp.j, bh_kv);
-              tma_prefetch_l2_4d(&tm_v, bx * BOXW, prow, wp.j, bh_kv);
-            }
+            tma_prefetch_l2_4d(&tm_k, bx * BOXW, p1, p2, bh_kv);
+            tma_prefetch_l2_4d(&tm_v, bx * BOXW, p1, p2, bh_kv);
           }
           walk_next(g, wp, a_hi, BN);
         }
-        const int krow = w.kb * BN;
+        int c1, c2;
+        shard_map_coords(g, w.j, w.kb * BN, c1, c2);
         for (int kv = 0; kv < 2 && ok; ++kv, ++n) {
           const int slot = n % C::kSlots;
           const uint32_t ph = (uint32_t)(n / C::kSlots) & 1;
@@ -227,10 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const void* tm = kv == 0 ? static_cast<const void*>(&tm_k) : static_cast<const void*>(&tm_v);
           for (int bx = 0; bx < C::kBoxes; ++bx) {
             uint8_t* dst = smem + C::kOffKV + slot * C::kTileBytes + bx * C::kBoxBytes;
-            if (striped)
-              tma_load_4d(dst, tm, &full[slot], bx * BOXW, w.j, krow, bh_kv);
-            else
-              tma_load_4d(dst, tm, &full[slot], bx * BOXW, krow, w.j, bh_kv);
+            tma_load_4d(dst, tm, &full[slot], bx * BOXW, c1, c2, bh_kv);
           }
         }
         if (!ok) break;

@@ -154,7 +154,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int64_t a_hi = (a0 + BQ - 1 < g.Sq - 1) ? a0 + BQ - 1 : g.Sq - 1;
   const int bh_q = U.b * g.Hq + U.h;
   const int bh_kv = U.b * g.Hkv + U.h / (g.Hq / g.Hkv);
-  const bool striped = g.layout == kStriped;
 
   if (warp >= 8) {
     regs_decrease<kRegsOther>();
@@ -169,12 +168,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (ok && leader) mbar_arrive_expect_tx(&bars[kQFull], kCtas * NQ * kQTileBytes);
       for (int q = 0; q < NQ && ok; ++q) {
         const int row = (int)(a0 + 256 * q + 128 * rank);
+        int c1, c2;
+        shard_map_coords(g, U.i, row, c1, c2);
         for (int bx = 0; bx < 2; ++bx) {
           uint8_t* dst = smem + kOffQ + q * kQTileBytes + bx * kQBoxBytes;
-          if (striped)
-            tma_load_4d_2sm(dst, &tm_q, leader_q, bx * BOXW, U.i, row, bh_q);
-          else
-            tma_load_4d_2sm(dst, &tm_q, leader_q, bx * BOXW, row, U.i, bh_q);
+          tma_load_4d_2sm(dst, &tm_q, leader_q, bx * BOXW, c1, c2, bh_q);
         }
       }
       for (TileWalk w = walk_begin(g, U.i, a_hi, BN, p.s_begin, p.s_end); walk_valid(w) && ok;
@@ -188,20 +186,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           uint8_t* dst = smem + kOffKV + slot * kHalfBytes;
           if (kv == 0) {
             // K half: keys [64 r, 64 r + 64) of the tile, all 128 dims (two 64-dim boxes)
-            const int krow = w.kb * BN + 64 * (int)rank;
-            for (int bx = 0; bx < 2; ++bx) {
-              if (striped)
-                tma_load_4d_2sm(dst + bx * kKBoxBytes, &tm_k, leader_full, bx * BOXW, w.j, krow, bh_kv);
-              else
-                tma_load_4d_2sm(dst + bx * kKBoxBytes, &tm_k, leader_full, bx * BOXW, krow, w.j, bh_kv);
-            }
+            int c1, c2;
+            shard_map_coords(g, w.j, w.kb * BN + 64 * (int)rank, c1, c2);
+            for (int bx = 0; bx < 2; ++bx)
+              tma_load_4d_2sm(dst + bx * kKBoxBytes, &tm_k, leader_full, bx * BOXW, c1, c2, bh_kv);
           } else {
             // V half: all 128 keys of the tile, dims [64 r, 64 r + 64)
-            const int vrow = w.kb * BN;
-            if (striped)
-              tma_load_4d_2sm(dst, &tm_v, leader_full, 64 * (int)rank, w.j, vrow, bh_kv);
-            else
-              tma_load_4d_2sm(dst, &tm_v, leader_full, 64 * (int)rank, vrow, w.j, bh_kv);
+            int c1, c2;
+            shard_map_coords(g, w.j, w.kb * BN, c1, c2);
+            tma_load_4d_2sm(dst, &tm_v, leader_full, 64 * (int)rank, c1, c2, bh_kv);
           }
         }
       }

@@ -8,6 +8,10 @@
 //   section 7 "causal attention with striped attention": under a causal mask
 //     token t sees only tokens u <= t (inclusive diagonal); the striped layout
 //     deals tokens round-robin, token t on shard t mod P.
+// RingAttention newsletter (cmlonder), section "claim and reality": striped or
+//   zigzag schedules balance the causal ring. Zigzag is named there without a
+//   definition; the reading used here cuts the sequence into 2P chunks of
+//   C = S/(2P) tokens and gives shard i chunks i and 2P-1-i, in that order.
 //
 // On one GPU the ring becomes the order in which a work unit visits KV tiles.
 // Everything here is plain integer arithmetic, compiled for both host and device
@@ -24,21 +28,44 @@
 
 namespace ringattn {
 
-enum Layout : int { kContiguous = 0, kStriped = 1 };
+enum Layout : int { kContiguous = 0, kStriped = 1, kZigzag = 2 };
 
 struct RingGeom {
   int B, Hq, Hkv;
   int64_t S;
   int D, P;
   int causal;   // 0 | 1
-  int layout;   // kContiguous | kStriped
+  int layout;   // kContiguous | kStriped | kZigzag
   int64_t Sq;   // S / P
 };
 
 // Global token of local index a in shard i.
-//   contiguous: shard i = tokens [i*Sq, (i+1)*Sq); striped: token a*P + i.
+//   contiguous: shard i = tokens [i*Sq, (i+1)*Sq); striped: token a*P + i;
+//   zigzag: a < C is token i*C + a, a >= C is token (2P-1-i)*C + (a - C).
 RA_HD int64_t token_of(const RingGeom& g, int i, int64_t a) {
-  return g.layout == kStriped ? a * g.P + i : (int64_t)i * g.Sq + a;
+  if (g.layout == kStriped) return a * g.P + i;
+  if (g.layout == kZigzag) {
+    const int64_t C = g.Sq / 2;
+    return a < C ? (int64_t)i * C + a : (int64_t)(2 * g.P - 1 - i) * C + (a - C);
+  }
+  return (int64_t)i * g.Sq + a;
+}
+
+// Coordinates (dim 1, dim 2) of local row a of shard i in the layout's 4-D tensor
+// map; dim 0 is the head dimension and dim 3 batch*heads (see encode_shard_map).
+// Rows past the end of a shard land outside the map and are zero-filled by TMA.
+RA_HD void shard_map_coords(const RingGeom& g, int i, int64_t a, int& c1, int& c2) {
+  if (g.layout == kStriped) {
+    c1 = i;
+    c2 = (int)a;
+  } else if (g.layout == kZigzag) {
+    const int64_t C = g.Sq / 2;
+    c1 = (int)(a < C ? a : a - C);
+    c2 = a < C ? i : 2 * g.P - 1 - i;
+  } else {
+    c1 = (int)a;
+    c2 = i;
+  }
 }
 
 // KV shard met by query shard i at ring step s (0 <= s < P).
@@ -51,12 +78,22 @@ RA_HD int ring_step_of(int i, int j, int P) { return (i - j + P) % P; }
 // the local indices b < key_limit(g, i, j, a) (always further capped at Sq).
 //   contiguous causal: j < i all keys; j == i keys b <= a; j > i none.
 //   striped causal: token b*P+j <= a*P+i  <=>  b < a, or b == a and j <= i.
+//   zigzag causal: shard j's tokens rise with b (its first chunk precedes its
+//     second), so the visible keys are those of each chunk up to token t.
 RA_HD int64_t key_limit(const RingGeom& g, int i, int j, int64_t a) {
   int64_t lim;
   if (!g.causal) {
     lim = g.Sq;
   } else if (g.layout == kContiguous) {
     lim = (j < i) ? g.Sq : (j == i ? a + 1 : 0);
+  } else if (g.layout == kZigzag) {
+    const int64_t C = g.Sq / 2;
+    const int64_t t = token_of(g, i, a);
+    int64_t lo = t - (int64_t)j * C + 1;
+    int64_t hi = t - (int64_t)(2 * g.P - 1 - j) * C + 1;
+    lo = lo < 0 ? 0 : (lo > C ? C : lo);
+    hi = hi < 0 ? 0 : (hi > C ? C : hi);
+    lim = lo + hi;
   } else {
     lim = (j <= i) ? a + 1 : a;
   }
@@ -75,6 +112,8 @@ RA_HD int kv_tiles_for(const RingGeom& g, int i, int j, int64_t a_hi, int TK) {
 // launched in index order approximates longest-processing-time scheduling:
 //   contiguous causal: cost grows with i*nkt + (rows of tb), so order by the
 //     combined index c = i*nblk + tb, descending;
+//   zigzag causal with whole blocks per chunk: cost grows with the block's global
+//     position, so walk the 2P chunks from the last to the first;
 //   otherwise (striped causal, non-causal): cost depends on tb only, so order by
 //     tb descending; inside a tb the unit index runs over (b, kv head, i, head in
 //     the GQA group) so concurrently running units share K/V through L2.
@@ -101,6 +140,21 @@ RA_HD Unit decode_unit(const RingGeom& g, int BQ, int q_shard_only, int64_t u) {
     r.b = (int)(bh / g.Hq);
     r.h = (int)(bh % g.Hq);
     r.i = q_shard_only;
+    return r;
+  }
+  if (g.causal && g.layout == kZigzag && (g.Sq / 2) % BQ == 0) {
+    // zigzag causal: cost grows with the global position of the block; walk the 2P
+    // chunks from the last backwards (chunk c belongs to shard c or 2P-1-c)
+    const int64_t bh_n = (int64_t)g.B * g.Hq;
+    const int64_t nbc = nblk / 2;  // blocks per chunk
+    const int64_t pos = (int64_t)g.P * nblk - 1 - u / bh_n;
+    const int c = (int)(pos / nbc);
+    r.i = c < g.P ? c : 2 * g.P - 1 - c;
+    r.tb = (int)((c < g.P ? 0 : nbc) + pos % nbc);
+    int64_t bh = u % bh_n;
+    int64_t bg = bh / rep;
+    r.b = (int)(bg / g.Hkv);
+    r.h = (int)((bg % g.Hkv) * rep + bh % rep);
     return r;
   }
   if (g.causal && g.layout == kContiguous) {

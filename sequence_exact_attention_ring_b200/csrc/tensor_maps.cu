@@ -20,12 +20,13 @@ static PFN_encodeTiled get_encode_fn() {
   return fn;
 }
 
-// 4-D view (D, local, shard, batch*heads) of a [B, H, S, D] bf16 tensor whose
-// sequence axis is split into P shards: contiguous shards are consecutive token
-// ranges, striped shards interleave with stride P. Dimensions are listed
-// innermost first so the strides grow: the striped map lists the shard before the
-// local index and kernels swap those two coordinates for it. Box: 64 elements
-// (128 bytes, 128-byte swizzle) by `box_rows` tokens of one shard.
+// 4-D view of a [B, H, S, D] bf16 tensor whose sequence axis is split into P
+// shards, dimensions listed innermost first so the strides grow:
+//   contiguous (D, local, shard, batch*heads): shards are consecutive token ranges;
+//   striped    (D, shard, local, batch*heads): shards interleave with stride P;
+//   zigzag     (D, offset, chunk, batch*heads): 2P chunks of Sq/2 tokens.
+// shard_map_coords gives a row's (dim 1, dim 2). Box: 64 elements (128 bytes,
+// 128-byte swizzle) by `box_rows` consecutive tokens.
 int encode_shard_map(CUtensorMap* map, const void* base, const RingGeom& g, int heads, int D, int box_rows) {
   PFN_encodeTiled enc = get_encode_fn();
   if (!enc) return RING_ATTN_ECUDA;
@@ -38,6 +39,11 @@ int encode_shard_map(CUtensorMap* map, const void* base, const RingGeom& g, int 
     dims[0] = D; dims[1] = g.P; dims[2] = g.Sq; dims[3] = (uint64_t)g.B * heads;
     strides[0] = row; strides[1] = row * g.P; strides[2] = row * g.S;
     box[0] = 64; box[1] = 1; box[2] = box_rows; box[3] = 1;
+  } else if (g.layout == kZigzag) {
+    const uint64_t C = (uint64_t)g.Sq / 2;
+    dims[0] = D; dims[1] = C; dims[2] = 2 * (uint64_t)g.P; dims[3] = (uint64_t)g.B * heads;
+    strides[0] = row; strides[1] = row * C; strides[2] = row * g.S;
+    box[0] = 64; box[1] = box_rows; box[2] = 1; box[3] = 1;
   } else {
     dims[0] = D; dims[1] = g.Sq; dims[2] = g.P; dims[3] = (uint64_t)g.B * heads;
     strides[0] = row; strides[1] = row * g.Sq; strides[2] = row * g.S;

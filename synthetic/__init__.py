@@ -46,7 +46,7 @@ class Workload:
     D: int
     P: int
     causal: bool
-    layout: str         # "contiguous" | "striped"
+    layout: str         # "contiguous" | "striped" | "zigzag"
     seed: int
     heavy_keys: bool = False
     gen_device: str = "cpu"   # "cpu" or "cuda": where the seeded draw happens
@@ -101,6 +101,10 @@ WORKLOADS = {
     "c5_bf16_s1m_striped": Workload("c5_bf16_s1m_striped", "bf16", 1, 8, 8, 1048576, 128, 32, True,
                                     "striped", 4, gen_device="cuda",
                                     description="bf16 S=1048576 P=32 causal striped"),
+    # the 1M workload's shape under the zigzag layout (chunks of 16384 tokens)
+    "z5_bf16_s1m_zigzag": Workload("z5_bf16_s1m_zigzag", "bf16", 1, 8, 8, 1048576, 128, 32, True,
+                                   "zigzag", 7, gen_device="cuda",
+                                   description="bf16 S=1048576 P=32 causal zigzag"),
     # profiling stand-in: the 1M workload's shape at 1/8 the length (inputs 0.4 GB > L2,
     # ~45 ms per launch) so an ncu capture of every section ends in a minute or two
     "prof_bf16_s128k_striped": Workload("prof_bf16_s128k_striped", "bf16", 1, 8, 8, 131072, 128, 32, True,
@@ -156,6 +160,11 @@ def shard_boundary_rows(w: Workload) -> list[tuple[int, int, int]]:
         if w.layout == "contiguous":
             ts.add(i * Sq)
             ts.add(i * Sq + Sq - 1)
+        elif w.layout == "zigzag":  # shard i holds chunks i and 2P-1-i of C = Sq/2 tokens
+            C = Sq // 2
+            for c in (i, 2 * w.P - 1 - i):
+                ts.add(c * C)
+                ts.add(c * C + C - 1)
         else:  # striped: shard i holds tokens a*P + i
             ts.add(i)
             ts.add((Sq - 1) * w.P + i)

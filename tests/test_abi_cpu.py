@@ -68,7 +68,8 @@ def fwd(scale=0.1, **kw):
 @pytest.mark.parametrize("bad,code", [
     (dict(B=0), B.EINVAL), (dict(Hq=0), B.EINVAL), (dict(S=0), B.EINVAL), (dict(P=0), B.EINVAL),
     (dict(S=1000, P=3), B.EINVAL), (dict(Hq=3, Hkv=2), B.EINVAL), (dict(causal=2), B.EINVAL),
-    (dict(layout=5), B.EINVAL), (dict(dtype=7), B.EINVAL), (dict(D=96), B.EUNSUPPORTED),
+    (dict(layout=5), B.EINVAL), (dict(layout=2, S=1020), B.EINVAL), (dict(dtype=7), B.EINVAL),
+    (dict(D=96), B.EUNSUPPORTED),
     (dict(D=256), B.EUNSUPPORTED), (dict(q=0), B.EINVAL), (dict(lse=0), B.EINVAL),
     (dict(k=FAKE + 8), B.EALIGN), (dict(out=FAKE + 2), B.EALIGN), (dict(ws=0), B.EWORKSPACE),
     (dict(wsb=16), B.EWORKSPACE), (dict(scale=0.0), B.EINVAL), (dict(scale=-1.0), B.EINVAL),
@@ -107,10 +108,13 @@ def visit_counts(S, P, causal, layout, tq, tk):
 
 
 @pytest.mark.parametrize("S,P", [(8, 1), (8, 2), (24, 3), (24, 8), (64, 4), (96, 8), (256, 8), (512, 16)])
-@pytest.mark.parametrize("layout", [0, 1])
+@pytest.mark.parametrize("layout", [0, 1, 2])
 @pytest.mark.parametrize("causal", [0, 1])
 @pytest.mark.parametrize("tiles", [(4, 4), (8, 2), (6, 5), (256, 128), (64, 32)])
 def test_schedule_visits_every_allowed_pair_exactly_once(lib, S, P, layout, causal, tiles):
+    if layout == 2 and S % (2 * P):
+        assert B.ring_attn_debug_visit_counts(S, P, causal, layout, *tiles, np.zeros(1, np.int32).ctypes.data) < 0
+        return
     counts, _ = visit_counts(S, P, causal, layout, *tiles)
     t = np.arange(S)[:, None]
     u = np.arange(S)[None, :]
@@ -128,7 +132,8 @@ def unit_table(Bz, Hq, Hkv, S, P, causal, layout, tq=256):
 
 
 @pytest.mark.parametrize("cfg", [(1, 8, 8, 16384, 8, 1, 0), (1, 8, 8, 16384, 8, 1, 1), (2, 32, 8, 131072, 16, 1, 1),
-                                 (1, 2, 2, 1024, 4, 0, 0), (1, 4, 1, 4096, 4, 1, 0), (1, 8, 8, 1 << 20, 32, 1, 1)])
+                                 (1, 2, 2, 1024, 4, 0, 0), (1, 4, 1, 4096, 4, 1, 0), (1, 8, 8, 1 << 20, 32, 1, 1),
+                                 (1, 8, 8, 16384, 8, 1, 2), (2, 8, 2, 65536, 16, 1, 2), (1, 8, 8, 1 << 20, 32, 1, 2)])
 def test_units_cover_each_block_once_longest_first(lib, cfg):
     Bz, Hq, Hkv, S, P, causal, layout = cfg
     tab = unit_table(Bz, Hq, Hkv, S, P, causal, layout)
@@ -148,13 +153,17 @@ def test_gqa_group_members_are_adjacent_in_launch_order(lib):
         assert sorted(x[1] % 4 for x in grp) == [0, 1, 2, 3]
 
 
-@pytest.mark.parametrize("layout", [0, 1])
+@pytest.mark.parametrize("layout", [0, 1, 2])
 @pytest.mark.parametrize("causal", [0, 1])
 def test_unit_walk_follows_ring_order(lib, layout, causal):
     S, P = 4096, 8
+    names = {0: "contiguous", 1: "striped", 2: "zigzag"}
     tab = unit_table(1, 1, 1, S, P, causal, layout)
     for u in range(len(tab)):
         i = tab[u, 2]
+        # the unit's last row sees the most keys; shards it cannot see at all are skipped
+        a_hi = min(tab[u, 3] * 256 + 255, S // P - 1)
+        t_hi = oracle.shard_tokens(S, P, names[layout], i)[a_hi]
         pairs = np.zeros((4096, 2), dtype=np.int32)
         n = B.ring_attn_debug_unit_walk(1, 1, 1, S, P, causal, layout, 256, 128, u, pairs.ctypes.data, 4096)
         assert n == tab[u, 4]
@@ -162,8 +171,8 @@ def test_unit_walk_follows_ring_order(lib, layout, causal):
         # ring step s meets kv shard (i - s) mod P: visiting order of distinct shards
         order = [shards[0]] + [s for a, s in zip(shards[:-1], shards[1:]) if s != a]
         expect = [(i - s) % P for s in range(P)]
-        if causal and layout == 0:
-            expect = [j for j in expect if j <= i]
+        if causal:
+            expect = [j for j in expect if oracle.shard_tokens(S, P, names[layout], j).min() <= t_hi]
         assert order == expect
         assert order[0] == i
         # inside one shard the key tiles run 0, 1, 2, ...

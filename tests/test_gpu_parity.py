@@ -34,6 +34,14 @@ SMALL = [
     (1, 2, 2, 1100, 128, 1, True, "contiguous", "bf16", "tcgen05"),    # ragged tail inside a 512-row pair block
     (1, 3, 3, 640, 128, 2, True, "striped", "bf16", "simt"),
     (1, 2, 2, 384, 64, 4, False, "contiguous", "bf16", "simt"),
+    # zigzag: shard i = chunks i and 2P-1-i of C = S/(2P) tokens
+    (1, 2, 2, 2048, 128, 4, True, "zigzag", "bf16", "tcgen05"),      # C=256: 512-row units span two chunks
+    (2, 4, 2, 3072, 128, 3, True, "zigzag", "bf16", "tcgen05"),      # C=512: chunk-ordered units, GQA 2
+    (1, 2, 2, 1024, 128, 4, False, "zigzag", "bf16", "tcgen05"),     # C=128, non-causal
+    (1, 4, 4, 2560, 64, 5, True, "zigzag", "bf16", "tcgen05"),       # D=64
+    (1, 2, 2, 2048, 128, 4, True, "zigzag", "bf16", "tcgen05_1sm"),
+    (1, 2, 2, 1000, 128, 4, True, "zigzag", "bf16", "auto"),         # C=125: AUTO takes the SIMT kernel
+    (1, 2, 2, 640, 64, 4, True, "zigzag", "fp32", "auto"),
 ]
 
 
@@ -75,7 +83,7 @@ def test_layouts_and_kernels_agree(cuda_lib):
     """Layout and kernel choice only change the schedule: outputs agree with each other."""
     base = (1, 4, 2, 2048, 128, 8, True)
     res = {}
-    for layout in ("contiguous", "striped"):
+    for layout in ("contiguous", "striped", "zigzag"):
         for algo in ("tcgen05", "tcgen05_1sm", "simt"):
             _, _, _, _, out, lse = run_case(*base, layout, "bf16", algo, seed=77)
             res[(layout, algo)] = (out.float(), lse)
@@ -85,7 +93,16 @@ def test_layouts_and_kernels_agree(cuda_lib):
         assert ((l - ref_l).abs() / ref_l.abs().clamp_min(1)).max().item() <= 1e-3, key
 
 
-@pytest.mark.parametrize("name", ["c4_bf16_gqa_s128k", "c5_bf16_s1m_striped"])
+def test_zigzag_chunks_the_tensor_cores_cannot_tile_are_refused(cuda_lib):
+    from sequence_exact_attention_ring_b200 import binding
+    w = synthetic.custom("zz", "bf16", 1, 2, 2, 1000, 128, 4, True, "zigzag", 1)
+    q, k, v = (t.cuda() for t in synthetic.make_inputs(w, "cpu"))
+    with pytest.raises(binding.RingAttnError) as e:
+        ring_attention(q, k, v, w.P, True, "zigzag", w.scale, algo="tcgen05")
+    assert e.value.code == binding.EUNSUPPORTED
+
+
+@pytest.mark.parametrize("name", ["c4_bf16_gqa_s128k", "c5_bf16_s1m_striped", "z5_bf16_s1m_zigzag"])
 def test_large_configs_sampled_rows(cuda_lib, name):
     """Full-size launch (as the benchmark runs it), checked on 4096 seeded rows + shard boundaries."""
     w = synthetic.get(name)

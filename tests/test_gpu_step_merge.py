@@ -13,10 +13,11 @@ pytestmark = pytest.mark.gpu
 
 @pytest.mark.parametrize("algo,dtype", [("tcgen05", "bf16"), ("tcgen05_1sm", "bf16"), ("simt", "bf16"),
                                         ("simt", "fp32")])
-@pytest.mark.parametrize("layout", ["contiguous", "striped"])
+@pytest.mark.parametrize("layout", ["contiguous", "striped", "zigzag"])
 def test_ring_steps_merged_equal_full_forward(cuda_lib, algo, dtype, layout):
     """Device i's P ring steps (one literal block each), merged, give the fused result."""
-    B, Hq, Hkv, S, D, P = 1, 2, 2, 1152, 128, 4
+    B, Hq, Hkv, D, P = 1, 2, 2, 128, 4
+    S = 2048 if layout == "zigzag" else 1152
     w = synthetic.custom("steps", dtype, B, Hq, Hkv, S, D, P, True, layout, 5)
     q, k, v = (t.cuda() for t in synthetic.make_inputs(w, "cpu"))
     O_ref, L_ref = oracle.attention_reference(q.cpu(), k.cpu(), v.cpu(), True, w.scale)

@@ -179,15 +179,41 @@ def test_rows_and_full_agree():
 def test_shard_maps():
     np.testing.assert_array_equal(oracle.shard_tokens(12, 3, "contiguous", 1), [4, 5, 6, 7])
     np.testing.assert_array_equal(oracle.shard_tokens(12, 3, "striped", 1), [1, 4, 7, 10])
-    for layout in ("contiguous", "striped"):
+    # zigzag: 2P chunks of S/(2P) tokens, shard i holds chunks i and 2P-1-i
+    np.testing.assert_array_equal(oracle.shard_tokens(16, 2, "zigzag", 0), [0, 1, 2, 3, 12, 13, 14, 15])
+    np.testing.assert_array_equal(oracle.shard_tokens(16, 2, "zigzag", 1), [4, 5, 6, 7, 8, 9, 10, 11])
+    for layout in ("contiguous", "striped", "zigzag"):
         allt = np.concatenate([oracle.shard_tokens(24, 4, layout, i) for i in range(4)])
         np.testing.assert_array_equal(np.sort(allt), np.arange(24))
     with pytest.raises(ValueError):
         oracle.shard_tokens(10, 3, "striped", 0)
+    with pytest.raises(ValueError):
+        oracle.shard_tokens(12, 4, "zigzag", 0)  # S % 2P != 0
+
+
+def _causal_pairs_per_shard(S, P, layout):
+    """(query, key) pairs each query shard folds under the causal mask, over all ring steps."""
+    counts = []
+    for i in range(P):
+        tq = oracle.shard_tokens(S, P, layout, i)
+        counts.append(sum(int(oracle.block_allowed(tq, oracle.shard_tokens(S, P, layout, j), True).sum())
+                          for j in range(P)))
+    return counts
+
+
+@pytest.mark.parametrize("S,P", [(16, 2), (48, 4), (64, 8)])
+def test_causal_work_per_shard_closed_forms(S, P):
+    """Contiguous: shard i folds i full blocks and one triangle, i*Sq^2 + Sq(Sq+1)/2 pairs.
+    Zigzag: chunks i and 2P-1-i together see 2P-1 full chunks and two triangles,
+    (2P-1)C^2 + C(C+1) pairs for every shard, so the ring is balanced."""
+    Sq, C = S // P, S // (2 * P)
+    assert _causal_pairs_per_shard(S, P, "contiguous") == [i * Sq * Sq + Sq * (Sq + 1) // 2 for i in range(P)]
+    assert _causal_pairs_per_shard(S, P, "zigzag") == [(2 * P - 1) * C * C + C * (C + 1)] * P
+    assert sum(_causal_pairs_per_shard(S, P, "striped")) == S * (S + 1) // 2
 
 
 @pytest.mark.parametrize("P", [1, 2, 4, 8])
-@pytest.mark.parametrize("layout", ["contiguous", "striped"])
+@pytest.mark.parametrize("layout", ["contiguous", "striped", "zigzag"])
 @pytest.mark.parametrize("causal", [False, True])
 def test_online_ring_equals_full_softmax(P, layout, causal):
     q, k, v = qkv(1, 4, 2, 32, 8, seed=61 + P)
@@ -200,7 +226,7 @@ def test_online_ring_equals_full_softmax(P, layout, causal):
 def test_online_ring_heavy_logits_no_nan():
     q, k, v = qkv(1, 2, 2, 32, 8, seed=71)
     k = k * 30.0
-    for layout in ("contiguous", "striped"):
+    for layout in ("contiguous", "striped", "zigzag"):
         O1, L1 = oracle.attention_reference(q, k, v, True, 1.0)
         O2, L2 = oracle.ring_attention_online(q, k, v, 8, True, layout, 1.0)
         assert np.isfinite(O2).all() and np.isfinite(L2).all()
@@ -269,8 +295,10 @@ def _pins_pass():
         test_uniform_keys_give_mean_of_allowed_values(True)
         test_single_dominant_key_returns_its_value(False)
         test_gqa_equals_mha_with_repeated_kv()
-        for layout in ("contiguous", "striped"):
+        for layout in ("contiguous", "striped", "zigzag"):
             test_online_ring_equals_full_softmax(4, layout, True)
+        test_shard_maps()
+        test_causal_work_per_shard_closed_forms(48, 4)
         test_merge_two_parts_closed_form()
     except (AssertionError, FloatingPointError, ValueError, IndexError):
         return False
@@ -282,7 +310,7 @@ def test_pins_pass_on_the_real_oracle():
 
 
 @pytest.mark.parametrize("mistake", ["exclusive_diagonal", "no_max_subtraction", "wrong_gqa_map",
-                                     "striped_transposed", "merge_no_weight"])
+                                     "striped_transposed", "zigzag_shifted_pairing", "merge_no_weight"])
 def test_planted_mistakes_fail_a_pin(monkeypatch, mistake):
     if mistake == "exclusive_diagonal":
         monkeypatch.setattr(oa, "allowed_keys",
@@ -302,6 +330,18 @@ def test_planted_mistakes_fail_a_pin(monkeypatch, mistake):
             # local index and shard index swapped: i*P + a instead of a*P + i
             return (i * P + np.arange(S // P)) if layout == "striped" else t
         monkeypatch.setattr(oa, "shard_tokens", bad)
+    elif mistake == "zigzag_shifted_pairing":
+        real = oa.shard_tokens
+
+        def bad(S, P, layout, i):
+            if layout != "zigzag":
+                return real(S, P, layout, i)
+            # pairs chunk i with chunk P+i: still a partition, but not the balanced one
+            C = S // (2 * P)
+            c = np.arange(C)
+            return np.concatenate([i * C + c, (P + i) * C + c])
+        monkeypatch.setattr(oa, "shard_tokens", bad)
+        monkeypatch.setattr(oracle, "shard_tokens", bad)
     elif mistake == "merge_no_weight":
         def bad(o_parts, lse_parts):
             return np.mean(np.stack(o_parts), axis=0), np.log(np.sum(np.exp(np.stack(lse_parts)), axis=0))

@@ -16,3 +16,10 @@ from .attention import (  # noqa: F401
     shard_tokens,
     softmax_row,
 )
+from .backward import (  # noqa: F401
+    attention_backward_reference,
+    backward_rows_dkdv,
+    backward_rows_dq,
+    delta_rows,
+    ring_attention_backward_online,
+)

@@ -130,6 +130,36 @@ int ring_attn_merge(const float* o_parts, const float* lse_parts, int n_parts, i
                     void* out, float* lse_out, int out_dtype, void* stream);
 
 /*
+ * Bytes of device workspace ring_attn_bwd needs: the 256-byte status header plus two
+ * fp32 arrays of B*Hq*P*ceil(S/P / 128)*128 values (per-row statistics in shard order).
+ * Returns 0 for invalid arguments.
+ */
+size_t ring_attn_bwd_workspace_bytes(int B, int Hq, int Hkv, int64_t S, int D, int P,
+                                     int causal, int layout, int dtype);
+
+/*
+ * Backward pass of ring_attn_fwd (RingAttention deep-architecture article, section
+ * "activation checkpointing and memory recomputation": only Q and the row statistics
+ * are kept, and K/V travel the ring in the opposite direction while the attention map
+ * is recomputed). Given the forward's out and lse and the output gradient dout, it
+ * writes the gradients of out with respect to q, k and v:
+ *   P = exp(scale q k^T - lse) on the mask,  dv = P^T dout,  dP = dout v^T,
+ *   Delta = rowsum(dout * out),  dS = P * (dP - Delta),
+ *   dq = scale dS k,  dk = scale dS^T q   (GQA: dk, dv sum over the group's heads).
+ *   q, out, dout, dq : device [B,Hq,S,D] bf16       k, v, dk, dv : device [B,Hkv,S,D] bf16
+ *   lse              : device [B,Hq,S] fp32 as returned by ring_attn_fwd
+ *   workspace        : >= ring_attn_bwd_workspace_bytes(); first word is the status word
+ * Supported: dtype bf16, D = 128, an sm_100 device (zigzag needs (S/(2P)) % 128 == 0);
+ * otherwise RING_ATTN_EUNSUPPORTED. Outputs must not alias inputs. Same argument
+ * and watchdog rules as ring_attn_fwd.
+ */
+int ring_attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                  const void* dout, void* dq, void* dk, void* dv,
+                  int B, int Hq, int Hkv, int64_t S, int D, int P,
+                  int causal, int layout, float scale, int dtype,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Synchronise `stream` and read the status word at the start of `workspace`
  * (written by the last compute call that used it): 0, or RING_ATTN_ETIMEOUT.
  * Returns RING_ATTN_ECUDA if the stream reports an error.
@@ -168,6 +198,16 @@ int ring_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* out
                           void* stream, void** scratch_out);
 
 /* ---- test hooks ------------------------------------------------------------ */
+
+/*
+ * Host only, no GPU. Walks the exact schedule and per-element masks of one pass of
+ * ring_attn_bwd (pass 0: the dK/dV kernel's KV units and the query tiles each meets;
+ * pass 1: the dQ kernel's query units and their backward-ring walk) with 128-row
+ * tiles and adds 1 to counts[t*S + u] for every (query token t, key token u) pair
+ * it lets into the gradient. counts: host S*S int32 zeroed by the caller, S <= 4096.
+ * Returns the number of tile visits, or a negative error code.
+ */
+int64_t ring_attn_debug_bwd_visit_counts(int64_t S, int P, int causal, int layout, int pass, int32_t* counts);
 
 /*
  * Host only, no GPU. Walks the exact unit/tile schedule and per-element masks the

@@ -90,6 +90,35 @@ def ring_attention_step(q, k, v, P: int, q_shard: int, kv_shard: int, causal: bo
     return o, lse
 
 
+def ring_attention_backward(q, k, v, out, lse, dout, P: int, causal: bool = True, layout="striped",
+                            scale: float | None = None, workspace=None, stream=None):
+    """Gradients (dq, dk, dv) of ring_attention's output against dout, from its out and lse.
+
+    bf16 tensors, D = 128. Asynchronous on `stream`.
+    """
+    _check_qkv(q, k, v)
+    for t, name in ((out, "out"), (dout, "dout")):
+        if t.shape != q.shape or t.dtype != q.dtype or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor shaped and typed like q")
+    B, Hq, S, D = q.shape
+    if lse.shape != (B, Hq, S) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 [B, Hq, S] tensor")
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    wsb = _b.ring_attn_bwd_workspace_bytes(B, Hq, k.shape[1], S, D, P, int(causal), _layout(layout),
+                                           _DTYPES[q.dtype])
+    if wsb == 0:
+        raise _b.RingAttnError(_b.EINVAL, "ring_attn_bwd_workspace_bytes")
+    if workspace is None or workspace.numel() < wsb:
+        workspace = torch.empty(wsb, dtype=torch.uint8, device=q.device)
+    rc = _b.ring_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), dout.data_ptr(),
+                          dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, k.shape[1], S, D, P, int(causal),
+                          _layout(layout), scale, _DTYPES[q.dtype], workspace.data_ptr(), workspace.numel(),
+                          _stream_ptr(stream))
+    _b.check(rc, "ring_attn_bwd")
+    return dq, dk, dv
+
+
 def merge(o_parts: torch.Tensor, lse_parts: torch.Tensor, out_dtype=torch.float32, stream=None):
     """Merge normalised partials o_parts [n, ..., D] fp32 / lse_parts [n, ...] -> (out [..., D], lse [...])."""
     if o_parts.dtype != torch.float32 or lse_parts.dtype != torch.float32:

@@ -46,6 +46,11 @@ SIGNATURES = {
                                     _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _c_int, _vp, _c_size, _vp]),
     "ring_attn_merge": (_c_int, [_vp, _vp, _c_int, _c_i64, _c_int, _vp, _vp, _c_int, _vp]),
     "ring_attn_status": (_c_int, [_vp, _vp]),
+    "ring_attn_bwd_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int, _c_i64, _c_int, _c_int, _c_int, _c_int,
+                                                _c_int]),
+    "ring_attn_bwd": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_i64, _c_int,
+                               _c_int, _c_int, _c_int, _c_float, _c_int, _vp, _c_size, _vp]),
+    "ring_attn_debug_bwd_visit_counts": (_c_i64, [_c_i64, _c_int, _c_int, _c_int, _c_int, _vp]),
     "ring_attn_fwd_noalloc": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_i64, _c_int, _c_int,
                                        _c_int, _c_int, _c_float, _c_int, _vp, ctypes.POINTER(_vp)]),
     "ring_attn_debug_visit_counts": (_c_i64, [_c_i64, _c_int, _c_int, _c_int, _c_int, _c_int, _vp]),
@@ -131,6 +136,20 @@ def ring_attn_merge(o_parts, lse_parts, n_parts, rows, D, out, lse_out, out_dtyp
 
 def ring_attn_status(workspace, stream) -> int:
     return load().ring_attn_status(workspace, stream)
+
+
+def ring_attn_bwd_workspace_bytes(B, Hq, Hkv, S, D, P, causal, layout, dtype) -> int:
+    return load().ring_attn_bwd_workspace_bytes(B, Hq, Hkv, S, D, P, causal, layout, dtype)
+
+
+def ring_attn_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, Hq, Hkv, S, D, P, causal, layout, scale, dtype, workspace,
+                  workspace_bytes, stream) -> int:
+    return load().ring_attn_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, Hq, Hkv, S, D, P, causal, layout, scale,
+                                dtype, workspace, workspace_bytes, stream)
+
+
+def ring_attn_debug_bwd_visit_counts(S, P, causal, layout, pass_, counts) -> int:
+    return load().ring_attn_debug_bwd_visit_counts(S, P, causal, layout, pass_, counts)
 
 
 def ring_attn_fwd_noalloc(q, k, v, out, lse, B, Hq, Hkv, S, D, P, causal, layout, scale, dtype, stream):

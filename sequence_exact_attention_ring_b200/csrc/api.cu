@@ -183,6 +183,35 @@ int ring_attn_merge(const float* o_parts, const float* lse_parts, int n_parts, i
                       static_cast<cudaStream_t>(stream));
 }
 
+size_t ring_attn_bwd_workspace_bytes(int B, int Hq, int Hkv, int64_t S, int D, int P, int causal, int layout,
+                                     int dtype) {
+  RingGeom g;
+  if (check_geom(B, Hq, Hkv, S, D, P, causal, layout, dtype, &g) != RING_ATTN_OK) return 0;
+  return kWorkspaceHeaderBytes + 2 * sizeof(float) * (size_t)B * Hq * P * (size_t)bwd_sq_pad(g);
+}
+
+int ring_attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dout,
+                  void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int64_t S, int D, int P, int causal,
+                  int layout, float scale, int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  RingGeom g;
+  int rc = check_geom(B, Hq, Hkv, S, D, P, causal, layout, dtype, &g);
+  if (rc) return rc;
+  if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv) return RING_ATTN_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return RING_ATTN_EALIGN;
+  const size_t need = ring_attn_bwd_workspace_bytes(B, Hq, Hkv, S, D, P, causal, layout, dtype);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return RING_ATTN_EWORKSPACE;
+  if (!(scale > 0.f) || !isfinite(scale)) return RING_ATTN_EINVAL;
+  if (dtype != RING_ATTN_DTYPE_BF16 || D != 128 || !tcgen05_layout_ok(g) || !device_is_sm100())
+    return RING_ATTN_EUNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((rc = reset_status(workspace, st))) return rc;
+  float* stats = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kWorkspaceHeaderBytes);
+  return launch_bwd_sm100(q, k, v, out, lse, dout, dq, dk, dv, g, scale, stats, static_cast<int*>(workspace),
+                          watchdog_ns(), st);
+}
+
 int ring_attn_status(const void* workspace, void* stream) {
   if (!workspace) return RING_ATTN_EINVAL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -190,6 +219,53 @@ int ring_attn_status(const void* workspace, void* stream) {
   int status = 0;
   if (cudaMemcpy(&status, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return RING_ATTN_ECUDA;
   return status;
+}
+
+int64_t ring_attn_debug_bwd_visit_counts(int64_t S, int P, int causal, int layout, int pass, int32_t* counts) {
+  RingGeom g;
+  int rc = check_geom(1, 1, 1, S, 128, P, causal, layout, RING_ATTN_DTYPE_BF16, &g);
+  if (rc) return rc;
+  if (!counts || S > 4096 || (pass != 0 && pass != 1)) return RING_ATTN_EINVAL;
+  const int T = 128;
+  int64_t visits = 0;
+  if (pass == 0) {
+    // dK/dV pass: every KV unit, every query tile it meets, the kernel's column rule
+    for (int64_t uu = 0; uu < num_kv_units(g, T); ++uu) {
+      const KvUnit U = decode_kv_unit(g, T, uu);
+      for (QWalk w = qwalk_begin(g, U, T, T); qwalk_valid(w); qwalk_next(g, w, T)) {
+        ++visits;
+        for (int r = 0; r < T; ++r) {
+          const int64_t b = (int64_t)U.kt * T + r;
+          if (b >= g.Sq) continue;
+          const int64_t u = token_of(g, U.j, b);
+          const int cmin = bwd_first_visible_col(g, w.i, (int64_t)w.qt * T, u, T);
+          for (int c = cmin; c < T; ++c) {
+            const int64_t a = (int64_t)w.qt * T + c;
+            if (a < g.Sq) counts[token_of(g, w.i, a) * S + u] += 1;
+          }
+        }
+      }
+    }
+  } else {
+    // dQ pass: every query unit, its backward-ring walk, the key limit per row
+    for (int64_t uu = 0; uu < num_units(g, T, -1); ++uu) {
+      const Unit U = decode_unit(g, T, -1, uu);
+      const int64_t a0 = (int64_t)U.tb * T;
+      const int64_t a_hi = (a0 + T - 1 < g.Sq - 1) ? a0 + T - 1 : g.Sq - 1;
+      for (TileWalk w = walk_begin_rev(g, U.i, a_hi, T); walk_valid(w); walk_next(g, w, a_hi, T)) {
+        ++visits;
+        for (int r = 0; r < T && a0 + r < g.Sq; ++r) {
+          const int64_t a = a0 + r;
+          const int64_t lim = key_limit(g, U.i, w.j, a);
+          for (int c = 0; c < T; ++c) {
+            const int64_t b = (int64_t)w.kb * T + c;
+            if (b < lim) counts[token_of(g, U.i, a) * S + token_of(g, w.j, b)] += 1;
+          }
+        }
+      }
+    }
+  }
+  return visits;
 }
 
 int64_t ring_attn_debug_visit_counts(int64_t S, int P, int causal, int layout, int tile_q, int tile_k,

@@ -1,0 +1,596 @@
+// Backward pass of exact ring attention for sm_100a (B200), D = 128, bf16 inputs.
+//
+// Method (RingAttention deep-architecture article, techknowgenie, section
+// "activation checkpointing and memory recomputation"): the forward keeps only the
+// queries and the row statistics; the backward lets the K/V blocks travel the ring
+// in the opposite direction and recomputes the attention map where they meet the
+// queries. The statistics are kept as lse = m + ln l, one number per row. With
+// S = scale Q K^T on the causal mask (global token order), the gradients of
+// O = softmax(S) V against dO are the chain rule through that definition:
+//     P = exp(S - lse),  dV = P^T dO,  dP = dO V^T,  Delta = rowsum(dO * O),
+//     dS = P * (dP - Delta),  dQ = scale dS K,  dK = scale dS^T Q.
+//
+// Three kernels, all on one stream:
+//   bwd_prep_kernel    Delta and lse * log2(e) per query row, written in shard-local
+//                      order and padded to whole 128-row tiles (+inf / 0 padding), so
+//                      a query tile's statistics are 512 contiguous bytes.
+//   bwd_dkdv_kernel    one CTA per K/V tile (b, kv head, shard j, 128 keys). As the
+//                      tile travels the backward ring it meets query shard (j - s) mod P
+//                      at step s; the CTA visits every query tile (of every query head
+//                      of the GQA group) that sees it:
+//                          S^T = K Q^T, dP^T = V dO^T        (SS MMAs into TMEM)
+//                          P^T, dS^T per key row              (8 warps, registers)
+//                          dV += P^T dO, dK += dS^T Q         (A operands from TMEM)
+//                      and writes dK, dV once, without atomics.
+//   bwd_dq_kernel      one CTA per query tile; it walks the K/V tiles in backward-ring
+//                      order (shard (i + s) mod P at step s):
+//                          S = Q K^T, dP = dO V^T, then P, dS per query row,
+//                          dQ += dS K                         (A operand from TMEM)
+// Splitting dQ from dK/dV recomputes S and dP once more (7 instead of 5 GEMMs) and
+// in exchange needs no atomic accumulation anywhere.
+//
+// Tensor memory (512 columns) in both main kernels: the transposed or plain score
+// tile [0,128), the dP tile [128,256), accumulators from 256. Eight elementwise
+// warps split each tile: warp w owns TMEM lanes 32 (w % 4) .. +31 and columns
+// 64 (w / 4) .. +63 of the score and dP tiles; it writes its 64 bf16 P (or dS)
+// values packed into the first 32 of those columns. Each 32-column chunk is read
+// before its 16 packed columns are stored, and chunk c's packed columns overlap only
+// chunk 0's fp32 columns, so no value is overwritten before it is read.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "ring_schedule.h"
+#include "ringattn_internal.h"
+#include "sm100_ptx.cuh"
+#include "softmax_rows.cuh"
+
+namespace ringattn {
+namespace bwd {
+
+constexpr int D = 128;
+constexpr int BT = 128;                    // rows of every tile (keys or queries)
+constexpr int BOXW = 64;                   // bf16 per TMA box row (128 bytes, 128B swizzle)
+constexpr int kBoxBytes = BT * BOXW * 2;   // 16 KiB
+constexpr int kTileBytes = BT * D * 2;     // 32 KiB
+constexpr int kStatBytes = BT * 4;         // 128 fp32 statistics of a query tile
+constexpr int kSmemLimit = 232448;
+constexpr int kThreads = 384;              // 8 elementwise warps, producer, MMA, 2 idle
+constexpr int kEwWarps = 8;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr uint32_t kProducerSleepNs = 64;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0;
+constexpr uint32_t kColDP = 128;
+constexpr uint32_t kColAcc = 256;
+constexpr uint32_t kIdescSS = idesc_bf16_f32(BT, BT, 0, 0);  // both operands K-major
+constexpr uint32_t kIdescTS = idesc_bf16_f32(BT, D, 0, 1);   // B MN-major (rows of the K dim)
+
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > limit_ns) return;
+  }
+}
+
+// K-major operand descriptor of a 128-row tile staged as two 64-column boxes; K
+// step k (16 columns) sits in box k/4 at byte 32 (k%4) of each 128-byte row.
+__device__ __forceinline__ uint64_t kmajor_step(uint64_t base, int k) {
+  return base + (uint64_t)((((k / 4) * kBoxBytes) + (k % 4) * 32) >> 4);
+}
+// MN-major operand (rows of the tile run along K): K step k covers rows 16k..16k+15.
+__device__ __forceinline__ uint64_t mnmajor_step(uint64_t base, int k) {
+  return base + (uint64_t)((k * 16 * 128) >> 4);
+}
+// TMEM column of K step k of a packed bf16 operand written by the two column halves.
+__device__ __forceinline__ uint32_t packed_step_col(int k) { return (uint32_t)((k / 4) * 64 + (k % 4) * 8); }
+
+// ----------------------------------------------------------------------- prep
+// One warp per padded shard-local query row (bh, i, a): lse2 = lse * log2(e) and
+// delta = <dO_t, O_t> in fp32 for t = token_of(i, a); rows a >= Sq get +inf and 0.
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const uint16_t* __restrict__ out,
+                                                       const uint16_t* __restrict__ dout,
+                                                       const float* __restrict__ lse, float* __restrict__ lse2,
+                                                       float* __restrict__ delta, RingGeom g, int64_t sq_pad,
+                                                       int64_t rows) {
+  const int64_t row = (int64_t)blockIdx.x * 8 + threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  if (row >= rows) return;
+  const int64_t per_bh = (int64_t)g.P * sq_pad;
+  const int64_t bh = row / per_bh;
+  const int i = (int)((row % per_bh) / sq_pad);
+  const int64_t a = row % sq_pad;
+  if (a >= g.Sq) {
+    if (lane == 0) {
+      lse2[row] = INFINITY;
+      delta[row] = 0.f;
+    }
+    return;
+  }
+  const int64_t t = token_of(g, i, a);
+  const int64_t base = (bh * g.S + t) * g.D;
+  float acc = 0.f;
+  for (int d = lane * 4; d < g.D; d += 128) {
+    const uint2 o = *reinterpret_cast<const uint2*>(out + base + d);
+    const uint2 x = *reinterpret_cast<const uint2*>(dout + base + d);
+    acc += __uint_as_float(o.x << 16) * __uint_as_float(x.x << 16);
+    acc += __uint_as_float(o.x & 0xffff0000u) * __uint_as_float(x.x & 0xffff0000u);
+    acc += __uint_as_float(o.y << 16) * __uint_as_float(x.y << 16);
+    acc += __uint_as_float(o.y & 0xffff0000u) * __uint_as_float(x.y & 0xffff0000u);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (lane == 0) {
+    lse2[row] = lse[bh * g.S + t] * 1.4426950408889634f;
+    delta[row] = acc;
+  }
+}
+
+struct Params {
+  RingGeom g;
+  const float* lse2;   // [B*Hq][P][sq_pad]
+  const float* delta;  // [B*Hq][P][sq_pad]
+  int64_t sq_pad;
+  void* out0;          // dK (dk/dv pass) or dQ (dq pass), bf16 [B,H,S,D]
+  void* out1;          // dV (dk/dv pass)
+  float scale;
+  float scale_log2;
+  int* status;
+  uint64_t watchdog_ns;
+};
+
+// P and dS for 32 columns: s, dp raw fp32 bits; stat_lse2/stat_delta per column (or
+// broadcast); columns c < cmin (or c >= cmax) are masked to P = 0.
+__device__ __forceinline__ void p_ds_chunk(const uint32_t (&s)[32], const uint32_t (&dp)[32], const float* lse2c,
+                                           const float* deltac, float row_lse2, float row_delta, bool per_col,
+                                           float scale_log2, int c0, int cmin, int cmax, uint32_t* pp,
+                                           uint32_t* pds) {
+#pragma unroll
+  for (int e = 0; e < 32; e += 2) {
+    float pv[2], dv[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int c = c0 + e + h;
+      const float l2 = per_col ? lse2c[e + h] : row_lse2;
+      const float dl = per_col ? deltac[e + h] : row_delta;
+      const bool on = c >= cmin && c < cmax;
+      const float x = fmaf(__uint_as_float(s[e + h]), scale_log2, -l2);
+      const float pe = on ? ex2_approx(x) : 0.f;
+      pv[h] = pe;
+      dv[h] = pe * (__uint_as_float(dp[e + h]) - dl);
+    }
+    pp[e / 2] = pack_bf16x2(pv[0], pv[1]);
+    pds[e / 2] = pack_bf16x2(dv[0], dv[1]);
+  }
+}
+
+// Shared memory of the dK/dV kernel: K and V tiles, then a ring of query-side slots
+// (a Q or dO tile followed by its 128 statistics).
+constexpr int kA_OffK = 0;
+constexpr int kA_OffV = kTileBytes;
+constexpr int kA_OffRing = 2 * kTileBytes;
+constexpr int kA_SlotBytes = ((kTileBytes + kStatBytes + 1023) / 1024) * 1024;
+constexpr int kA_Slots = (kSmemLimit - 1024 - 64 - 512 - kA_OffRing) / kA_SlotBytes;
+constexpr int kA_OffBar = kA_OffRing + kA_Slots * kA_SlotBytes;
+enum BarA { kA_KVFull = 0, kA_STFull = 1, kA_PReady = 2, kA_Done = 3, kA_Drain = 4, kA_Ring = 5 };
+constexpr int kA_NumBars = kA_Ring + 2 * kA_Slots;
+constexpr int kA_OffMisc = kA_OffBar + kA_NumBars * 8;
+constexpr int kA_SmemBytes = kA_OffMisc + 64 + 1024;
+static_assert(kA_Slots >= 2, "need a Q and a dO slot");
+static_assert(kA_SmemBytes <= kSmemLimit, "shared memory budget");
+
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                    const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kA_OffBar);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kA_OffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kA_OffMisc + 8);
+  uint64_t* full = &bars[kA_Ring];
+  uint64_t* empty = &bars[kA_Ring + kA_Slots];
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const RingGeom& g = p.g;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars[kA_KVFull], 1);
+    mbar_init(&bars[kA_STFull], 1);
+    mbar_init(&bars[kA_PReady], kEwWarps);
+    mbar_init(&bars[kA_Done], 1);
+    mbar_init(&bars[kA_Drain], 1);
+    for (int s = 0; s < 2 * kA_Slots; ++s) mbar_init(&bars[kA_Ring + s], 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const Watchdog wd{abort_flag, p.status, p.watchdog_ns};
+  const KvUnit U = decode_kv_unit(g, BT, blockIdx.x);
+  const int bh_kv = U.b * g.Hkv + U.g;
+  const int rep = g.Hq / g.Hkv;
+  const int64_t N = qwalk_count(g, U, BT, BT);  // query tiles met (x2 loads each)
+  auto slot_of = [&](int64_t m) { return (int)(m % kA_Slots); };
+  auto phase_of = [&](int64_t m) { return (uint32_t)((m / kA_Slots) & 1); };
+
+  if (warp == kProducerWarp) {
+    if (lane == 0 && N > 0) {
+      // ------------------------------------------------------------------ producer
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_do);
+      int c1, c2;
+      shard_map_coords(g, U.j, (int64_t)U.kt * BT, c1, c2);
+      mbar_arrive_expect_tx(&bars[kA_KVFull], 2 * kTileBytes);
+      for (int bx = 0; bx < 2; ++bx) {
+        tma_load_4d(smem + kA_OffK + bx * kBoxBytes, &tm_k, &bars[kA_KVFull], bx * BOXW, c1, c2, bh_kv);
+        tma_load_4d(smem + kA_OffV + bx * kBoxBytes, &tm_v, &bars[kA_KVFull], bx * BOXW, c1, c2, bh_kv);
+      }
+      int64_t m = 0;
+      bool ok = true;
+      for (QWalk w = qwalk_begin(g, U, BT, BT); qwalk_valid(w) && ok; qwalk_next(g, w, BT)) {
+        const int bh_q = U.b * g.Hq + U.g * rep + w.hr;
+        const int64_t a0 = (int64_t)w.qt * BT;
+        shard_map_coords(g, w.i, a0, c1, c2);
+        const int64_t stat = ((int64_t)bh_q * g.P + w.i) * p.sq_pad + a0;
+        for (int kind = 0; kind < 2; ++kind, ++m) {
+          const int slot = slot_of(m);
+          if (!(ok = mbar_wait_backoff<false>(&empty[slot], phase_of(m) ^ 1, wd, kProducerSleepNs))) break;
+          uint8_t* dst = smem + kA_OffRing + slot * kA_SlotBytes;
+          mbar_arrive_expect_tx(&full[slot], kTileBytes + kStatBytes);
+          const CUtensorMap* tm = kind == 0 ? &tm_q : &tm_do;
+          for (int bx = 0; bx < 2; ++bx) tma_load_4d(dst + bx * kBoxBytes, tm, &full[slot], bx * BOXW, c1, c2, bh_q);
+          bulk_load(dst + kTileBytes, (kind == 0 ? p.lse2 : p.delta) + stat, kStatBytes, &full[slot]);
+        }
+      }
+      if (!ok) {
+        // wind down: this CTA's own copies must land before its shared memory goes away
+        drain_wait(&bars[kA_KVFull], 0, p.watchdog_ns);
+        for (int64_t x = (m > kA_Slots ? m - kA_Slots : 0); x < m; ++x)
+          drain_wait(&full[slot_of(x)], phase_of(x), p.watchdog_ns);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------------ MMA issuer
+    const bool issuer = elect_one_sync();
+    const uint32_t sbase = smem_u32(smem);
+    const uint64_t dK = smem_desc_sw128(sbase + kA_OffK, 0, 1024);
+    const uint64_t dV = smem_desc_sw128(sbase + kA_OffV, 0, 1024);
+    auto all = [&](bool r) { return __all_sync(0xffffffffu, r); };
+    bool ok = N > 0 && all(mbar_wait(&bars[kA_KVFull], 0, wd));
+    for (int64_t n = 0; ok && n < N; ++n) {
+      const int sq = slot_of(2 * n), sd = slot_of(2 * n + 1);
+      const uint32_t aq = sbase + kA_OffRing + sq * kA_SlotBytes;
+      const uint32_t ad = sbase + kA_OffRing + sd * kA_SlotBytes;
+      if (!(ok = all(mbar_wait(&full[sq], phase_of(2 * n), wd)))) break;
+      if (!(ok = all(mbar_wait(&full[sd], phase_of(2 * n + 1), wd)))) break;
+      tc_fence_after();
+      const uint64_t bq = smem_desc_sw128(aq, 0, 1024), bd = smem_desc_sw128(ad, 0, 1024);
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k)
+        if (issuer) mma_ss(tmem + kColS, kmajor_step(dK, k), kmajor_step(bq, k), kIdescSS, k > 0);
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k)
+        if (issuer) mma_ss(tmem + kColDP, kmajor_step(dV, k), kmajor_step(bd, k), kIdescSS, k > 0);
+      if (issuer) mma_commit(&bars[kA_STFull]);
+      if (!(ok = all(mbar_wait(&bars[kA_PReady], (uint32_t)(n & 1), wd)))) break;
+      tc_fence_after();
+      const uint64_t mq = smem_desc_sw128(aq, kBoxBytes, 1024), md = smem_desc_sw128(ad, kBoxBytes, 1024);
+#pragma unroll
+      for (int k = 0; k < BT / 16; ++k)  // dV += P^T dO
+        if (issuer) mma_ts(tmem + kColAcc, tmem + kColS + packed_step_col(k), mnmajor_step(md, k), kIdescTS,
+                           !(n == 0 && k == 0));
+#pragma unroll
+      for (int k = 0; k < BT / 16; ++k)  // dK += dS^T Q
+        if (issuer) mma_ts(tmem + kColAcc + D, tmem + kColDP + packed_step_col(k), mnmajor_step(mq, k), kIdescTS,
+                           !(n == 0 && k == 0));
+      if (issuer) {
+        mma_commit(&empty[sq]);
+        mma_commit(&empty[sd]);
+      }
+    }
+    if (issuer) {
+      mma_commit(&bars[kA_Done]);
+      mma_commit(&bars[kA_Drain]);
+    }
+    drain_wait(&bars[kA_Drain], 0, p.watchdog_ns);
+  } else if (warp < kEwWarps) {
+    // ------------------------------------------------------------- elementwise + epilogue
+    const int wq = warp % 4, hh = warp / 4;
+    const int r = wq * 32 + lane;
+    const int64_t b = (int64_t)U.kt * BT + r;  // key row of shard j
+    const int64_t u = token_of(g, U.j, b);
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_off + kColS + hh * 64;
+    const uint32_t tDP = tmem + lane_off + kColDP + hh * 64;
+    int64_t n = 0;
+    bool ok = true;
+    int row_i = -1;       // query shard of the cached first visible row
+    int64_t row0 = 0;     // first row of shard row_i whose token is >= u
+    for (QWalk w = qwalk_begin(g, U, BT, BT); qwalk_valid(w); qwalk_next(g, w, BT), ++n) {
+      const int sq = slot_of(2 * n), sd = slot_of(2 * n + 1);
+      if (!(ok = mbar_wait(&bars[kA_STFull], (uint32_t)(n & 1), wd))) break;
+      // the statistics came with the tiles: wait on their barriers too (already complete)
+      if (!(ok = mbar_wait(&full[sq], phase_of(2 * n), wd) && mbar_wait(&full[sd], phase_of(2 * n + 1), wd))) break;
+      tc_fence_after();
+      const float* lse2c = reinterpret_cast<const float*>(smem + kA_OffRing + sq * kA_SlotBytes + kTileBytes);
+      const float* deltac = reinterpret_cast<const float*>(smem + kA_OffRing + sd * kA_SlotBytes + kTileBytes);
+      if (w.i != row_i) {
+        row_i = w.i;
+        row0 = g.causal ? first_row_at_or_after(g, w.i, u) : 0;
+      }
+      const int64_t cm = row0 - (int64_t)w.qt * BT;
+      const int cmin = cm < 0 ? 0 : (cm > BT ? BT : (int)cm);
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t s[32], dp[32], pp[16], pds[16];
+        tmem_ld32(tS + cc * 32, s);
+        tmem_ld32(tDP + cc * 32, dp);
+        tmem_wait_ld();
+        const int c0 = hh * 64 + cc * 32;
+        p_ds_chunk(s, dp, lse2c + c0, deltac + c0, 0.f, 0.f, true, p.scale_log2, c0, cmin, BT, pp, pds);
+        tmem_st16(tS + cc * 16, pp);
+        tmem_st16(tDP + cc * 16, pds);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[kA_PReady]);
+    }
+    const bool have = n > 0 && ok && mbar_wait(&bars[kA_Done], 0, wd);
+    if (have || n == 0) {
+      tc_fence_after();
+      const bool row_ok = b < g.Sq;
+      const int64_t out_row = (int64_t)bh_kv * g.S + (row_ok ? u : 0);
+      const uint32_t tAcc = tmem + lane_off + kColAcc + hh * 64;
+      store_row_cols<64>(tAcc, n > 0, row_ok, 1.f, false, p.out1, out_row, D, hh * 64);         // dV
+      store_row_cols<64>(tAcc + D, n > 0, row_ok, p.scale, false, p.out0, out_row, D, hh * 64);  // dK
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// Shared memory of the dQ kernel: Q and dO once, then a ring of K/V tile slots.
+constexpr int kB_OffQ = 0;
+constexpr int kB_OffDO = kTileBytes;
+constexpr int kB_OffRing = 2 * kTileBytes;
+constexpr int kB_Slots = (kSmemLimit - 1024 - 64 - 512 - kB_OffRing) / kTileBytes;
+constexpr int kB_OffBar = kB_OffRing + kB_Slots * kTileBytes;
+enum BarB { kB_QFull = 0, kB_SFull = 1, kB_PReady = 2, kB_Done = 3, kB_Drain = 4, kB_Ring = 5 };
+constexpr int kB_NumBars = kB_Ring + 2 * kB_Slots;
+constexpr int kB_OffMisc = kB_OffBar + kB_NumBars * 8;
+constexpr int kB_SmemBytes = kB_OffMisc + 64 + 1024;
+static_assert(kB_Slots >= 2, "need a K and a V slot");
+static_assert(kB_SmemBytes <= kSmemLimit, "shared memory budget");
+
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                  const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kB_OffBar);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kB_OffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kB_OffMisc + 8);
+  uint64_t* full = &bars[kB_Ring];
+  uint64_t* empty = &bars[kB_Ring + kB_Slots];
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const RingGeom& g = p.g;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars[kB_QFull], 1);
+    mbar_init(&bars[kB_SFull], 1);
+    mbar_init(&bars[kB_PReady], kEwWarps);
+    mbar_init(&bars[kB_Done], 1);
+    mbar_init(&bars[kB_Drain], 1);
+    for (int s = 0; s < 2 * kB_Slots; ++s) mbar_init(&bars[kB_Ring + s], 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const Watchdog wd{abort_flag, p.status, p.watchdog_ns};
+  const Unit U = decode_unit(g, BT, -1, blockIdx.x);
+  const int64_t a0 = (int64_t)U.tb * BT;
+  const int64_t a_hi = (a0 + BT - 1 < g.Sq - 1) ? a0 + BT - 1 : g.Sq - 1;
+  const int bh_q = U.b * g.Hq + U.h;
+  const int bh_kv = U.b * g.Hkv + U.h / (g.Hq / g.Hkv);
+  const int64_t N = unit_tile_count(g, U.i, a_hi, BT, 0, g.P);  // the same tiles in either ring direction
+  auto slot_of = [&](int64_t m) { return (int)(m % kB_Slots); };
+  auto phase_of = [&](int64_t m) { return (uint32_t)((m / kB_Slots) & 1); };
+
+  if (warp == kProducerWarp) {
+    if (lane == 0 && N > 0) {
+      // ------------------------------------------------------------------ producer
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      int c1, c2;
+      shard_map_coords(g, U.i, a0, c1, c2);
+      mbar_arrive_expect_tx(&bars[kB_QFull], 2 * kTileBytes);
+      for (int bx = 0; bx < 2; ++bx) {
+        tma_load_4d(smem + kB_OffQ + bx * kBoxBytes, &tm_q, &bars[kB_QFull], bx * BOXW, c1, c2, bh_q);
+        tma_load_4d(smem + kB_OffDO + bx * kBoxBytes, &tm_do, &bars[kB_QFull], bx * BOXW, c1, c2, bh_q);
+      }
+      int64_t m = 0;
+      bool ok = true;
+      for (TileWalk w = walk_begin_rev(g, U.i, a_hi, BT); walk_valid(w) && ok; walk_next(g, w, a_hi, BT)) {
+        shard_map_coords(g, w.j, (int64_t)w.kb * BT, c1, c2);
+        for (int kind = 0; kind < 2; ++kind, ++m) {
+          const int slot = slot_of(m);
+          if (!(ok = mbar_wait_backoff<false>(&empty[slot], phase_of(m) ^ 1, wd, kProducerSleepNs))) break;
+          uint8_t* dst = smem + kB_OffRing + slot * kTileBytes;
+          mbar_arrive_expect_tx(&full[slot], kTileBytes);
+          const CUtensorMap* tm = kind == 0 ? &tm_k : &tm_v;
+          for (int bx = 0; bx < 2; ++bx)
+            tma_load_4d(dst + bx * kBoxBytes, tm, &full[slot], bx * BOXW, c1, c2, bh_kv);
+        }
+      }
+      if (!ok) {
+        drain_wait(&bars[kB_QFull], 0, p.watchdog_ns);
+        for (int64_t x = (m > kB_Slots ? m - kB_Slots : 0); x < m; ++x)
+          drain_wait(&full[slot_of(x)], phase_of(x), p.watchdog_ns);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------------ MMA issuer
+    const bool issuer = elect_one_sync();
+    const uint32_t sbase = smem_u32(smem);
+    const uint64_t dQd = smem_desc_sw128(sbase + kB_OffQ, 0, 1024);
+    const uint64_t dOd = smem_desc_sw128(sbase + kB_OffDO, 0, 1024);
+    auto all = [&](bool r) { return __all_sync(0xffffffffu, r); };
+    bool ok = N > 0 && all(mbar_wait(&bars[kB_QFull], 0, wd));
+    for (int64_t n = 0; ok && n < N; ++n) {
+      const int sk = slot_of(2 * n), sv = slot_of(2 * n + 1);
+      const uint32_t ak = sbase + kB_OffRing + sk * kTileBytes;
+      const uint32_t av = sbase + kB_OffRing + sv * kTileBytes;
+      if (!(ok = all(mbar_wait(&full[sk], phase_of(2 * n), wd)))) break;
+      if (!(ok = all(mbar_wait(&full[sv], phase_of(2 * n + 1), wd)))) break;
+      tc_fence_after();
+      const uint64_t bk = smem_desc_sw128(ak, 0, 1024), bv = smem_desc_sw128(av, 0, 1024);
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k)  // S = Q K^T
+        if (issuer) mma_ss(tmem + kColS, kmajor_step(dQd, k), kmajor_step(bk, k), kIdescSS, k > 0);
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k)  // dP = dO V^T
+        if (issuer) mma_ss(tmem + kColDP, kmajor_step(dOd, k), kmajor_step(bv, k), kIdescSS, k > 0);
+      if (issuer) {
+        mma_commit(&bars[kB_SFull]);
+        mma_commit(&empty[sv]);  // V is no longer needed once dP is done
+      }
+      if (!(ok = all(mbar_wait(&bars[kB_PReady], (uint32_t)(n & 1), wd)))) break;
+      tc_fence_after();
+      const uint64_t mk = smem_desc_sw128(ak, kBoxBytes, 1024);
+#pragma unroll
+      for (int k = 0; k < BT / 16; ++k)  // dQ += dS K
+        if (issuer) mma_ts(tmem + kColAcc, tmem + kColS + packed_step_col(k), mnmajor_step(mk, k), kIdescTS,
+                           !(n == 0 && k == 0));
+      if (issuer) mma_commit(&empty[sk]);
+    }
+    if (issuer) {
+      mma_commit(&bars[kB_Done]);
+      mma_commit(&bars[kB_Drain]);
+    }
+    drain_wait(&bars[kB_Drain], 0, p.watchdog_ns);
+  } else if (warp < kEwWarps) {
+    // ------------------------------------------------------------- elementwise + epilogue
+    const int wq = warp % 4, hh = warp / 4;
+    const int r = wq * 32 + lane;
+    const int64_t a = a0 + r;
+    const int64_t stat = ((int64_t)bh_q * g.P + U.i) * p.sq_pad + a;  // a < sq_pad always
+    const float row_lse2 = p.lse2[stat];
+    const float row_delta = p.delta[stat];
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_off + kColS + hh * 64;
+    const uint32_t tDP = tmem + lane_off + kColDP + hh * 64;
+    int64_t n = 0;
+    bool ok = true;
+    for (TileWalk w = walk_begin_rev(g, U.i, a_hi, BT); walk_valid(w); walk_next(g, w, a_hi, BT), ++n) {
+      if (!(ok = mbar_wait(&bars[kB_SFull], (uint32_t)(n & 1), wd))) break;
+      tc_fence_after();
+      const int cut = visible_keys<BT>((int64_t)w.kb * BT, key_limit(g, U.i, w.j, a));
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t s[32], dp[32], pp[16], pds[16];
+        tmem_ld32(tS + cc * 32, s);
+        tmem_ld32(tDP + cc * 32, dp);
+        tmem_wait_ld();
+        const int c0 = hh * 64 + cc * 32;
+        p_ds_chunk(s, dp, nullptr, nullptr, row_lse2, row_delta, false, p.scale_log2, c0, 0, cut, pp, pds);
+        tmem_st16(tS + cc * 16, pds);  // only dS feeds the dQ MMA
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[kB_PReady]);
+    }
+    const bool have = n > 0 && ok && mbar_wait(&bars[kB_Done], 0, wd);
+    if (have || n == 0) {
+      tc_fence_after();
+      const bool row_ok = a < g.Sq;
+      const int64_t out_row = (int64_t)bh_q * g.S + (row_ok ? token_of(g, U.i, a) : 0);
+      store_row_cols<64>(tmem + lane_off + kColAcc + hh * 64, n > 0, row_ok, p.scale, false, p.out0, out_row, D,
+                         hh * 64);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace bwd
+
+int64_t bwd_sq_pad(const RingGeom& g) { return (g.Sq + bwd::BT - 1) / bwd::BT * bwd::BT; }
+
+int launch_bwd_sm100(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                     const void* dout, void* dq, void* dk, void* dv, const RingGeom& g, float scale, float* stats,
+                     int* status, uint64_t watchdog_ns, cudaStream_t stream) {
+  using namespace bwd;
+  if (g.D != D) return RING_ATTN_EUNSUPPORTED;
+  const int64_t sq_pad = bwd_sq_pad(g);
+  const int64_t rows = (int64_t)g.B * g.Hq * g.P * sq_pad;
+  float* lse2 = stats;
+  float* delta = stats + rows;
+  const int64_t prep_blocks = (rows + 7) / 8;
+  if (prep_blocks > 0x7fffffff) return RING_ATTN_EINVAL;
+  bwd_prep_kernel<<<(unsigned)prep_blocks, 256, 0, stream>>>(static_cast<const uint16_t*>(out),
+                                                              static_cast<const uint16_t*>(dout), lse, lse2, delta,
+                                                              g, sq_pad, rows);
+  if (cudaGetLastError() != cudaSuccess) return RING_ATTN_ECUDA;
+  CUtensorMap mq, mdo, mk, mv;
+  int rc;
+  if ((rc = encode_shard_map(&mq, q, g, g.Hq, D, BT)) != 0) return rc;
+  if ((rc = encode_shard_map(&mdo, dout, g, g.Hq, D, BT)) != 0) return rc;
+  if ((rc = encode_shard_map(&mk, k, g, g.Hkv, D, BT)) != 0) return rc;
+  if ((rc = encode_shard_map(&mv, v, g, g.Hkv, D, BT)) != 0) return rc;
+  Params p;
+  p.g = g;
+  p.lse2 = lse2;
+  p.delta = delta;
+  p.sq_pad = sq_pad;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.status = status;
+  p.watchdog_ns = watchdog_ns;
+  if (cudaFuncSetAttribute(bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kA_SmemBytes) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kB_SmemBytes) != cudaSuccess)
+    return RING_ATTN_ECUDA;
+  const int64_t kv_units = num_kv_units(g, BT);
+  const int64_t q_units = num_units(g, BT, -1);
+  if (kv_units > 0x7fffffff || q_units > 0x7fffffff) return RING_ATTN_EINVAL;
+  p.out0 = dk;
+  p.out1 = dv;
+  bwd_dkdv_kernel<<<(unsigned)kv_units, kThreads, kA_SmemBytes, stream>>>(mq, mdo, mk, mv, p);
+  if (cudaGetLastError() != cudaSuccess) return RING_ATTN_ECUDA;
+  p.out0 = dq;
+  p.out1 = nullptr;
+  bwd_dq_kernel<<<(unsigned)q_units, kThreads, kB_SmemBytes, stream>>>(mq, mdo, mk, mv, p);
+  return cudaGetLastError() == cudaSuccess ? RING_ATTN_OK : RING_ATTN_ECUDA;
+}
+
+}  // namespace ringattn

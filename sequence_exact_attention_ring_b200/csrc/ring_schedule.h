@@ -193,11 +193,12 @@ RA_HD int64_t unit_tile_count(const RingGeom& g, int i, int64_t a_hi, int TK, in
 struct TileWalk {
   int s, s_end, j, kb, nkb;
   int i, P;
+  int rev;  // 1: the backward ring, KV shard (i + s) mod P at step s
 };
 
 RA_HD void walk_skip_empty(const RingGeom& g, TileWalk& w, int64_t a_hi, int TK) {
   while (w.s < w.s_end) {
-    w.j = ring_kv_shard(w.i, w.s, g.P);
+    w.j = w.rev ? (w.i + w.s) % g.P : ring_kv_shard(w.i, w.s, g.P);
     w.nkb = kv_tiles_for(g, w.i, w.j, a_hi, TK);
     if (w.nkb > 0) return;
     ++w.s;
@@ -206,7 +207,18 @@ RA_HD void walk_skip_empty(const RingGeom& g, TileWalk& w, int64_t a_hi, int TK)
 
 RA_HD TileWalk walk_begin(const RingGeom& g, int i, int64_t a_hi, int TK, int s_begin, int s_end) {
   TileWalk w;
-  w.s = s_begin; w.s_end = s_end; w.i = i; w.P = g.P; w.kb = 0; w.j = 0; w.nkb = 0;
+  w.s = s_begin; w.s_end = s_end; w.i = i; w.P = g.P; w.kb = 0; w.j = 0; w.nkb = 0; w.rev = 0;
+  walk_skip_empty(g, w, a_hi, TK);
+  return w;
+}
+
+// The same walk over the backward ring (RingAttention deep-architecture article,
+// techknowgenie, section "activation checkpointing and memory recomputation": KV
+// blocks travel the ring in the opposite direction), so query shard i meets KV
+// shard (i + s) mod P at step s.
+RA_HD TileWalk walk_begin_rev(const RingGeom& g, int i, int64_t a_hi, int TK) {
+  TileWalk w;
+  w.s = 0; w.s_end = g.P; w.i = i; w.P = g.P; w.kb = 0; w.j = 0; w.nkb = 0; w.rev = 1;
   walk_skip_empty(g, w, a_hi, TK);
   return w;
 }
@@ -218,6 +230,126 @@ RA_HD void walk_next(const RingGeom& g, TileWalk& w, int64_t a_hi, int TK) {
   w.kb = 0;
   ++w.s;
   walk_skip_empty(g, w, a_hi, TK);
+}
+
+// ---------------------------------------------------------------- backward, K/V side
+// The dK/dV pass gives each CTA one KV tile (b, kv head g, KV shard j, tile kt of
+// TK keys) and lets it meet every query tile that can see it, the way a KV block
+// meets the query shards as it travels the backward ring: at step s it sits with
+// query shard (j - s) mod P. Inside a shard, query rows see a key exactly when
+// their token is not below the key's (causal), and tokens rise with the local index.
+
+// First local row of shard i whose token is >= u (Sq if none): binary search on the
+// monotone token map.
+RA_HD int64_t first_row_at_or_after(const RingGeom& g, int i, int64_t u) {
+  int64_t lo = 0, hi = g.Sq;
+  while (lo < hi) {
+    const int64_t mid = (lo + hi) / 2;
+    if (token_of(g, i, mid) >= u) hi = mid; else lo = mid + 1;
+  }
+  return lo;
+}
+
+struct KvUnit {
+  int b, g, j, kt;
+};
+
+RA_HD int64_t num_kv_tiles(const RingGeom& g, int TK) { return (g.Sq + TK - 1) / TK; }
+
+RA_HD int64_t num_kv_units(const RingGeom& g, int TK) { return (int64_t)g.B * g.Hkv * g.P * num_kv_tiles(g, TK); }
+
+// Longest first: a KV tile's work grows as its first token falls, so units run
+// from the earliest tiles of the sequence to the latest (contiguous causal: shard
+// j, then tile; zigzag causal with whole tiles per chunk: chunk 0..2P-1, then tile;
+// otherwise tile, then shard). (b, kv head) is innermost.
+RA_HD KvUnit decode_kv_unit(const RingGeom& g, int TK, int64_t u) {
+  const int64_t nkt = num_kv_tiles(g, TK);
+  const int64_t bg_n = (int64_t)g.B * g.Hkv;
+  const int64_t pos = u / bg_n;
+  const int64_t bg = u % bg_n;
+  KvUnit r;
+  r.b = (int)(bg / g.Hkv);
+  r.g = (int)(bg % g.Hkv);
+  if (g.causal && g.layout == kContiguous) {
+    r.j = (int)(pos / nkt);
+    r.kt = (int)(pos % nkt);
+  } else if (g.causal && g.layout == kZigzag && (g.Sq / 2) % TK == 0) {
+    const int64_t tpc = nkt / 2;  // tiles per chunk
+    const int c = (int)(pos / tpc);
+    r.j = c < g.P ? c : 2 * g.P - 1 - c;
+    r.kt = (int)((c < g.P ? 0 : tpc) + pos % tpc);
+  } else {
+    r.kt = (int)(pos / g.P);
+    r.j = (int)(pos % g.P);
+  }
+  return r;
+}
+
+// Walk over (query head of the group, ring step, query tile) for one KV tile.
+struct QWalk {
+  int hr, rep;  // query head hr of the GQA group
+  int s, i;     // ring step and the query shard met there
+  int qt, nqt;  // current query tile and the shard's tile count
+  int qt0;      // first query tile of shard i that sees the KV tile
+  int j;
+  int64_t u_min;  // smallest key token of the tile
+};
+
+RA_HD void qwalk_skip_empty(const RingGeom& g, QWalk& w, int TQ) {
+  while (w.hr < w.rep) {
+    while (w.s < g.P) {
+      w.i = (w.j - w.s + g.P) % g.P;
+      const int64_t a0 = g.causal ? first_row_at_or_after(g, w.i, w.u_min) : 0;
+      if (a0 < g.Sq) {
+        w.qt0 = (int)(a0 / TQ);
+        w.qt = w.qt0;
+        return;
+      }
+      ++w.s;
+    }
+    w.s = 0;
+    ++w.hr;
+  }
+}
+
+RA_HD QWalk qwalk_begin(const RingGeom& g, const KvUnit& U, int TQ, int TK) {
+  QWalk w;
+  w.hr = 0; w.rep = g.Hq / g.Hkv; w.s = 0; w.i = U.j; w.j = U.j;
+  w.nqt = (int)((g.Sq + TQ - 1) / TQ);
+  w.qt = 0; w.qt0 = 0;
+  w.u_min = token_of(g, U.j, (int64_t)U.kt * TK);
+  qwalk_skip_empty(g, w, TQ);
+  return w;
+}
+
+RA_HD bool qwalk_valid(const QWalk& w) { return w.hr < w.rep; }
+
+RA_HD void qwalk_next(const RingGeom& g, QWalk& w, int TQ) {
+  if (++w.qt < w.nqt) return;
+  ++w.s;
+  qwalk_skip_empty(g, w, TQ);
+}
+
+// Causal mask inside one (query tile, KV tile) block of the dK/dV pass: the key of
+// token u is visible to the tile's query columns c >= the returned value (query
+// rows a0 + c of shard i); 0 when not causal.
+RA_HD int bwd_first_visible_col(const RingGeom& g, int i, int64_t a0, int64_t u, int TQ) {
+  if (!g.causal) return 0;
+  const int64_t c = first_row_at_or_after(g, i, u) - a0;
+  return c < 0 ? 0 : (c > TQ ? TQ : (int)c);
+}
+
+// Query tiles one KV unit meets: per shard, the tiles from the first that sees the
+// KV tile's smallest token to the end, for every query head of the group.
+RA_HD int64_t qwalk_count(const RingGeom& g, const KvUnit& U, int TQ, int TK) {
+  const int64_t nqt = (g.Sq + TQ - 1) / TQ;
+  const int64_t u_min = token_of(g, U.j, (int64_t)U.kt * TK);
+  int64_t n = 0;
+  for (int i = 0; i < g.P; ++i) {
+    const int64_t a0 = g.causal ? first_row_at_or_after(g, i, u_min) : 0;
+    if (a0 < g.Sq) n += nqt - a0 / TQ;
+  }
+  return n * (g.Hq / g.Hkv);
 }
 
 }  // namespace ringattn

@@ -38,6 +38,13 @@ int launch_fwd_simt(const void* q, const void* k, const void* v, void* out, floa
                     float scale, int dtype, int s_begin, int s_end, int q_shard_only, int partial,
                     cudaStream_t stream);
 
+// Backward pass (bf16, D = 128): the Delta / lse prep kernel, then the dK/dV and dQ
+// tcgen05 kernels. `stats` holds 2 * B*Hq*P*bwd_sq_pad(g) floats.
+int64_t bwd_sq_pad(const RingGeom& g);
+int launch_bwd_sm100(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                     const void* dout, void* dq, void* dk, void* dv, const RingGeom& g, float scale, float* stats,
+                     int* status, uint64_t watchdog_ns, cudaStream_t stream);
+
 int launch_merge(const float* o_parts, const float* lse_parts, int n_parts, int64_t rows, int D, void* out,
                  float* lse_out, int out_dtype, cudaStream_t stream);
 

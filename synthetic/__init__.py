@@ -32,7 +32,7 @@ from typing import Iterable
 
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "get", "make_inputs", "sample_rows", "shard_boundary_rows"]
+__all__ = ["Workload", "WORKLOADS", "get", "make_inputs", "make_dout", "sample_rows", "shard_boundary_rows"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -150,6 +150,17 @@ def make_inputs(w: Workload, device: str | torch.device | None = None):
                 k[b, gh, idx, :] *= 4.0
     dt = w.torch_dtype
     return q.to(dt).contiguous(), k.to(dt).contiguous(), v.to(dt).contiguous()
+
+
+def make_dout(w: Workload, device: str | torch.device | None = None) -> torch.Tensor:
+    """The output gradient for backward tests: i.i.d. N(0, 1) drawn in fp32 with seed
+    w.seed + 500 on ``device`` (default: the workload's gen_device), shaped like q and
+    rounded to the workload dtype."""
+    dev = torch.device(device if device is not None else w.gen_device)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(w.seed + 500)
+    d = torch.randn((w.B, w.Hq, w.S, w.D), generator=gen, device=dev, dtype=torch.float32)
+    return d.to(w.torch_dtype).contiguous()
 
 
 def shard_boundary_rows(w: Workload) -> list[tuple[int, int, int]]:

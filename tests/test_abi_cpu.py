@@ -192,3 +192,46 @@ def test_schedule_info_matches_closed_form_for_1m_striped(lib):
     assert longest == first == 32 * 256 and last == 32 * 2
     # partial tiles: the last two of every shard step of every unit
     assert partial == 8 * 32 * nblk * 32 * 2
+
+
+# ------------------------------------------------------------------ backward schedule
+
+@pytest.mark.parametrize("S,P,layout", [(256, 1, 0), (256, 2, 1), (768, 3, 0), (1024, 4, 1), (1024, 8, 0),
+                                        (1000, 8, 1), (2048, 4, 2), (1536, 3, 2), (3072, 3, 2)])
+@pytest.mark.parametrize("causal", [0, 1])
+@pytest.mark.parametrize("pass_", [0, 1])
+def test_backward_schedule_visits_every_allowed_pair_exactly_once(lib, S, P, layout, causal, pass_):
+    """dK/dV pass (KV tiles meeting query tiles) and dQ pass (backward-ring walk)."""
+    counts = np.zeros((S, S), dtype=np.int32)
+    n = B.ring_attn_debug_bwd_visit_counts(S, P, causal, layout, pass_, counts.ctypes.data)
+    assert n > 0
+    t = np.arange(S)[:, None]
+    u = np.arange(S)[None, :]
+    allowed = (u <= t) if causal else np.ones((S, S), dtype=bool)
+    np.testing.assert_array_equal(counts, allowed.astype(np.int32))
+
+
+def test_backward_workspace_and_argument_errors(lib):
+    # status header + two fp32 arrays of B*Hq*P*ceil(Sq/128)*128
+    assert B.ring_attn_bwd_workspace_bytes(1, 8, 8, 16384, 128, 8, 1, 1, 1) == 256 + 2 * 4 * 8 * 8 * 2048
+    assert B.ring_attn_bwd_workspace_bytes(1, 2, 2, 1000, 128, 8, 1, 1, 1) == 256 + 2 * 4 * 2 * 8 * 128
+    assert B.ring_attn_bwd_workspace_bytes(1, 8, 8, 16383, 128, 8, 1, 0, 1) == 0
+    args = [FAKE] * 9 + [1, 2, 2, 1024, 128, 4, 1, 1, 0.1, 1, FAKE, 1 << 20, None]
+    bad = list(args)
+    bad[12] = 1022  # S % P != 0
+    assert B.ring_attn_bwd(*bad) == B.EINVAL
+    bad = list(args)
+    bad[5] = 0  # dout null
+    assert B.ring_attn_bwd(*bad) == B.EINVAL
+    bad = list(args)
+    bad[6] = FAKE + 4  # dq misaligned
+    assert B.ring_attn_bwd(*bad) == B.EALIGN
+    bad = list(args)
+    bad[20] = 64  # workspace too small
+    assert B.ring_attn_bwd(*bad) == B.EWORKSPACE
+    bad = list(args)
+    bad[17] = -0.5  # scale
+    assert B.ring_attn_bwd(*bad) == B.EINVAL
+    bad = list(args)
+    bad[18] = 0  # fp32: no backward kernel
+    assert B.ring_attn_bwd(*bad) == B.EUNSUPPORTED

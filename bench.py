@@ -52,6 +52,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
+    ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd"],
+                    help="fwd: the forward hot path (the headline line); bwd: ring_attn_bwd on the same workload")
     return ap.parse_args()
 
 
@@ -362,12 +364,81 @@ def run_ours(args, world, rank, local):
     print(json.dumps(line))
 
 
+BWD_METRIC = "causal-adjusted attention backward TFLOP/s (10*D FLOPs per allowed pair), 1 GPU"
+
+
+def run_backward(args, world, rank, local):
+    """Times ring_attn_bwd (prep + dK/dV + dQ kernels) on the workload; out/lse from one
+    untimed forward. Algorithmic work: 5 matrix products per allowed (query, key) pair,
+    10*D FLOPs (the kernels recompute S and dP once more, which is not counted)."""
+    from sequence_exact_attention_ring_b200 import binding, ring_attention, ring_attention_backward
+    w = synthetic.get(args.workload)
+    binding.load()
+    dev = torch.device("cuda", local if world > 1 else 0)
+    w_rank = synthetic.custom(w.name, w.dtype, w.B, w.Hq, w.Hkv, w.S, w.D, w.P, w.causal, w.layout,
+                              w.seed + rank, w.heavy_keys, "cuda")
+    q, k, v = synthetic.make_inputs(w_rank, dev)
+    dout = synthetic.make_dout(w_rank, dev)
+    out, lse = ring_attention(q, k, v, w.P, w.causal, w.layout, w.scale)
+    wsb = binding.ring_attn_bwd_workspace_bytes(w.B, w.Hq, w.Hkv, w.S, w.D, w.P, int(w.causal),
+                                                {"contiguous": 0, "striped": 1, "zigzag": 2}[w.layout], 1)
+    ws = torch.zeros(wsb, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        return ring_attention_backward(q, k, v, out, lse, dout, w.P, w.causal, w.layout, w.scale, workspace=ws,
+                                       stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    sampler = ClockSampler(dev.index)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    st = binding.ring_attn_status(ws.data_ptr(), stream.cuda_stream)
+    elapsed = max_over_ranks(t0.elapsed_time(t1), world)
+    launch_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in ev), world)
+    flops = 2.5 * w.causal_flops()
+    alg = 2.5 * w.algorithmic_flops()
+    peaks, peak_src = measured_peaks()
+    peak = float(peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"])
+    achieved = alg / (launch_ms * 1e-3) / 1e12
+    clocks_all = gather_objects(clocks, world)
+    if rank != 0:
+        return
+    print(json.dumps({
+        "metric": BWD_METRIC, "value": flops * world * args.steps / (elapsed * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(workload_config(w), **{"pass": "bwd", "flops_per_step": flops}),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "peak_source": f"{peak_src} bf16_tflops_sustained",
+                     "kernel": "bwd_prep_kernel + bwd_dkdv_kernel + bwd_dq_kernel (one ring_attn_bwd call)"},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks_all[0] if world == 1 else {"per_rank": clocks_all},
+        "status": st,
+    }))
+
+
 def main():
     args = parse()
     world, rank, local = dist_setup(args)
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)
+        elif args.which == "bwd":
+            run_backward(args, world, rank, local)
         else:
             run_ours(args, world, rank, local)
     finally:

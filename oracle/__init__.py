@@ -23,3 +23,4 @@ from .backward import (  # noqa: F401
     delta_rows,
     ring_attention_backward_online,
 )
+from .decode import decode_reference, decode_split  # noqa: F401

@@ -52,8 +52,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
-    ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd"],
-                    help="fwd: the forward hot path (the headline line); bwd: ring_attn_bwd on the same workload")
+    ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd", "decode"],
+                    help="fwd: the forward hot path (the headline line); bwd: ring_attn_bwd on the same workload; "
+                         "decode: one decode step against the workload's K/V as the cache")
     return ap.parse_args()
 
 
@@ -431,6 +432,66 @@ def run_backward(args, world, rank, local):
     }))
 
 
+DECODE_METRIC = "decode step against a sharded KV cache: cache GB/s read, 1 GPU"
+
+
+def run_decode(args, world, rank, local):
+    """Times ring_attn_decode (split-KV kernel + merge) with the workload's K/V as the cache.
+    Algorithmic bytes per step: K and V read once, q read, out and lse written."""
+    from sequence_exact_attention_ring_b200 import binding, ring_attention_decode
+    w = synthetic.get(args.workload)
+    binding.load()
+    dev = torch.device("cuda", local if world > 1 else 0)
+    w_rank = synthetic.custom(w.name, w.dtype, w.B, w.Hq, w.Hkv, w.S, w.D, w.P, False, w.layout, w.seed + rank,
+                              w.heavy_keys, "cuda")
+    _, k, v = synthetic.make_inputs(w_rank, dev)
+    q1 = synthetic.make_decode_query(w_rank, dev)
+    lay = {"contiguous": 0, "striped": 1, "zigzag": 2}[w.layout]
+    ws = torch.zeros(binding.ring_attn_decode_workspace_bytes(w.B, w.Hq, w.Hkv, w.S, w.D, w.P, lay, 1),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    esz = 2
+    nbytes = 2 * w.B * w.Hkv * w.S * w.D * esz + 2 * w.B * w.Hq * w.D * esz + w.B * w.Hq * 4
+
+    def step():
+        return ring_attention_decode(q1, k, v, w.P, w.layout, w.scale, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    sampler = ClockSampler(dev.index)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    st = binding.ring_attn_status(ws.data_ptr(), stream.cuda_stream)
+    ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in ev), world)
+    peaks, peak_src = measured_peaks()
+    peak = float(peaks["hbm_gbs"])
+    achieved = nbytes / (ms * 1e-3) / 1e9
+    clocks_all = gather_objects(clocks, world)
+    if rank != 0:
+        return
+    print(json.dumps({
+        "metric": DECODE_METRIC, "value": achieved * world, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": dict({k_: v_ for k_, v_ in workload_config(w).items() if k_ != "flops_per_step"},
+                       **{"pass": "decode", "causal": False, "cache_bytes": nbytes,
+                          "l2": "cache larger than L2 (no flush)"}),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": None, "peak_source": f"{peak_src} hbm_gbs",
+                     "kernel": "decode_kernel + merge_kernel (one ring_attn_decode call)"},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks_all[0] if world == 1 else {"per_rank": clocks_all},
+        "status": st,
+    }))
+
+
 def main():
     args = parse()
     world, rank, local = dist_setup(args)
@@ -439,6 +500,8 @@ def main():
             run_reference(args, world, rank)
         elif args.which == "bwd":
             run_backward(args, world, rank, local)
+        elif args.which == "decode":
+            run_decode(args, world, rank, local)
         else:
             run_ours(args, world, rank, local)
     finally:

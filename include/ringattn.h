@@ -160,6 +160,29 @@ int ring_attn_bwd(const void* q, const void* k, const void* v, const void* out, 
                   void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Bytes of device workspace ring_attn_decode needs: the status header plus the
+ * split-KV partials (at most 1024 per row). Returns 0 for invalid arguments.
+ */
+size_t ring_attn_decode_workspace_bytes(int B, int Hq, int Hkv, int64_t S, int D, int P, int layout, int dtype);
+
+/*
+ * One decode step against a KV cache of S tokens kept in P ring shards (layout as in
+ * ring_attn_fwd). Each head has one new query row whose position follows every cached
+ * key, so it attends to all S keys (no mask): out = softmax(scale q k^T) v, and lse.
+ * (After a million-token prefill, each new token reads the whole cache: RingAttention
+ * newsletter, cmlonder, section "code and integration map".) The cache is read once,
+ * split across SMs by shard and chunk, and the normalised partials are combined by
+ * the merge of ring_attn_merge.
+ *   q   : device [B, Hq, D] bf16          k, v : device [B, Hkv, S, D] bf16
+ *   out : device [B, Hq, D] bf16          lse  : device [B, Hq] fp32
+ * Supported: bf16, D = 128, Hq/Hkv <= 16, an sm_100 device (zigzag needs
+ * (S/(2P)) % 128 == 0); otherwise RING_ATTN_EUNSUPPORTED. S % P == 0.
+ */
+int ring_attn_decode(const void* q, const void* k, const void* v, void* out, float* lse,
+                     int B, int Hq, int Hkv, int64_t S, int D, int P, int layout, float scale, int dtype,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Synchronise `stream` and read the status word at the start of `workspace`
  * (written by the last compute call that used it): 0, or RING_ATTN_ETIMEOUT.
  * Returns RING_ATTN_ECUDA if the stream reports an error.

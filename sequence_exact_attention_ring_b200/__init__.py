@@ -6,7 +6,8 @@ does not load the library; the first call does, and raises if it is missing.
 """
 from . import binding  # noqa: F401
 from .api import (  # noqa: F401
-    HostRunner, merge, ring_attention, ring_attention_backward, ring_attention_step, status, workspace_bytes)
+    HostRunner, merge, ring_attention, ring_attention_backward, ring_attention_decode, ring_attention_step, status,
+    workspace_bytes)
 from .binding import RingAttnError  # noqa: F401
 
 __all__ = ["binding", "ring_attention", "ring_attention_step", "merge", "status", "workspace_bytes",

@@ -119,6 +119,34 @@ def ring_attention_backward(q, k, v, out, lse, dout, P: int, causal: bool = True
     return dq, dk, dv
 
 
+def ring_attention_decode(q1, k, v, P: int, layout="striped", scale: float | None = None, workspace=None,
+                          stream=None):
+    """One decode step: q1 [B, Hq, D] (one new row per head) against the cache k, v [B, Hkv, S, D]
+    kept in P ring shards. Returns (out [B, Hq, D] bf16, lse [B, Hq] fp32). Asynchronous on `stream`."""
+    if q1.dim() != 3 or k.dim() != 4 or v.shape != k.shape:
+        raise ValueError("q1 must be [B, Hq, D] and k, v [B, Hkv, S, D]")
+    for t in (q1, k, v):
+        if not t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError("q1, k, v must be contiguous bf16 CUDA tensors")
+    B, Hq, D = q1.shape
+    Hkv, S = k.shape[1], k.shape[2]
+    if k.shape[0] != B or k.shape[3] != D:
+        raise ValueError("shape mismatch between q1 and the cache")
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    out = torch.empty_like(q1)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=q1.device)
+    wsb = _b.ring_attn_decode_workspace_bytes(B, Hq, Hkv, S, D, P, _layout(layout), _b.DTYPE_BF16)
+    if wsb == 0:
+        raise _b.RingAttnError(_b.EINVAL, "ring_attn_decode_workspace_bytes")
+    if workspace is None or workspace.numel() < wsb:
+        workspace = torch.empty(wsb, dtype=torch.uint8, device=q1.device)
+    rc = _b.ring_attn_decode(q1.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Hq, Hkv, S,
+                             D, P, _layout(layout), scale, _b.DTYPE_BF16, workspace.data_ptr(), workspace.numel(),
+                             _stream_ptr(stream))
+    _b.check(rc, "ring_attn_decode")
+    return out, lse
+
+
 def merge(o_parts: torch.Tensor, lse_parts: torch.Tensor, out_dtype=torch.float32, stream=None):
     """Merge normalised partials o_parts [n, ..., D] fp32 / lse_parts [n, ...] -> (out [..., D], lse [...])."""
     if o_parts.dtype != torch.float32 or lse_parts.dtype != torch.float32:

@@ -50,6 +50,9 @@ SIGNATURES = {
                                                 _c_int]),
     "ring_attn_bwd": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_i64, _c_int,
                                _c_int, _c_int, _c_int, _c_float, _c_int, _vp, _c_size, _vp]),
+    "ring_attn_decode_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int, _c_i64, _c_int, _c_int, _c_int, _c_int]),
+    "ring_attn_decode": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_i64, _c_int, _c_int, _c_int,
+                                  _c_float, _c_int, _vp, _c_size, _vp]),
     "ring_attn_debug_bwd_visit_counts": (_c_i64, [_c_i64, _c_int, _c_int, _c_int, _c_int, _vp]),
     "ring_attn_fwd_noalloc": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_i64, _c_int, _c_int,
                                        _c_int, _c_int, _c_float, _c_int, _vp, ctypes.POINTER(_vp)]),
@@ -146,6 +149,16 @@ def ring_attn_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, Hq, Hkv, S, D, P, caus
                   workspace_bytes, stream) -> int:
     return load().ring_attn_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, Hq, Hkv, S, D, P, causal, layout, scale,
                                 dtype, workspace, workspace_bytes, stream)
+
+
+def ring_attn_decode_workspace_bytes(B, Hq, Hkv, S, D, P, layout, dtype) -> int:
+    return load().ring_attn_decode_workspace_bytes(B, Hq, Hkv, S, D, P, layout, dtype)
+
+
+def ring_attn_decode(q, k, v, out, lse, B, Hq, Hkv, S, D, P, layout, scale, dtype, workspace, workspace_bytes,
+                     stream) -> int:
+    return load().ring_attn_decode(q, k, v, out, lse, B, Hq, Hkv, S, D, P, layout, scale, dtype, workspace,
+                                   workspace_bytes, stream)
 
 
 def ring_attn_debug_bwd_visit_counts(S, P, causal, layout, pass_, counts) -> int:

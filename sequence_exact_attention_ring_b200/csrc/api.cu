@@ -212,6 +212,34 @@ int ring_attn_bwd(const void* q, const void* k, const void* v, const void* out, 
                           watchdog_ns(), st);
 }
 
+size_t ring_attn_decode_workspace_bytes(int B, int Hq, int Hkv, int64_t S, int D, int P, int layout, int dtype) {
+  RingGeom g;
+  if (check_geom(B, Hq, Hkv, S, D, P, 0, layout, dtype, &g) != RING_ATTN_OK) return 0;
+  const size_t rows = (size_t)B * Hq;
+  return kWorkspaceHeaderBytes + sizeof(float) * (size_t)decode_parts(g) * rows * (size_t)(D + 1);
+}
+
+int ring_attn_decode(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv,
+                     int64_t S, int D, int P, int layout, float scale, int dtype, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+  RingGeom g;
+  int rc = check_geom(B, Hq, Hkv, S, D, P, 0, layout, dtype, &g);
+  if (rc) return rc;
+  if (!q || !k || !v || !out || !lse) return RING_ATTN_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse)) return RING_ATTN_EALIGN;
+  const size_t need = ring_attn_decode_workspace_bytes(B, Hq, Hkv, S, D, P, layout, dtype);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return RING_ATTN_EWORKSPACE;
+  if (!(scale > 0.f) || !isfinite(scale)) return RING_ATTN_EINVAL;
+  if (dtype != RING_ATTN_DTYPE_BF16 || D != 128 || Hq / Hkv > 16 || !tcgen05_layout_ok(g) || !device_is_sm100())
+    return RING_ATTN_EUNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((rc = reset_status(workspace, st))) return rc;
+  float* o_parts = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kWorkspaceHeaderBytes);
+  float* lse_parts = o_parts + (size_t)decode_parts(g) * B * Hq * D;
+  return launch_decode_sm100(q, k, v, out, lse, g, scale, o_parts, lse_parts, static_cast<int*>(workspace),
+                             watchdog_ns(), st);
+}
+
 int ring_attn_status(const void* workspace, void* stream) {
   if (!workspace) return RING_ATTN_EINVAL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -45,6 +45,14 @@ int launch_bwd_sm100(const void* q, const void* k, const void* v, const void* ou
                      const void* dout, void* dq, void* dk, void* dv, const RingGeom& g, float scale, float* stats,
                      int* status, uint64_t watchdog_ns, cudaStream_t stream);
 
+// Decode (one query row per head against the whole sharded cache, bf16, D = 128):
+// split-KV partials into o_parts [decode_parts(g)][B*Hq][D] and lse_parts, then the
+// merge kernel writes out [B*Hq][D] bf16 and lse [B*Hq].
+int64_t decode_parts(const RingGeom& g);
+int launch_decode_sm100(const void* q, const void* k, const void* v, void* out, float* lse, const RingGeom& g,
+                        float scale, float* o_parts, float* lse_parts, int* status, uint64_t watchdog_ns,
+                        cudaStream_t stream);
+
 int launch_merge(const float* o_parts, const float* lse_parts, int n_parts, int64_t rows, int D, void* out,
                  float* lse_out, int out_dtype, cudaStream_t stream);
 

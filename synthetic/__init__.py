@@ -32,7 +32,7 @@ from typing import Iterable
 
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "get", "make_inputs", "make_dout", "sample_rows", "shard_boundary_rows"]
+__all__ = ["Workload", "WORKLOADS", "get", "make_inputs", "make_dout", "make_decode_query", "sample_rows", "shard_boundary_rows"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -161,6 +161,17 @@ def make_dout(w: Workload, device: str | torch.device | None = None) -> torch.Te
     gen.manual_seed(w.seed + 500)
     d = torch.randn((w.B, w.Hq, w.S, w.D), generator=gen, device=dev, dtype=torch.float32)
     return d.to(w.torch_dtype).contiguous()
+
+
+def make_decode_query(w: Workload, device: str | torch.device | None = None) -> torch.Tensor:
+    """One new query row per head for a decode step against the workload's K/V cache:
+    i.i.d. N(0, 1) drawn in fp32 with seed w.seed + 700, shape [B, Hq, D], rounded to
+    the workload dtype."""
+    dev = torch.device(device if device is not None else w.gen_device)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(w.seed + 700)
+    q1 = torch.randn((w.B, w.Hq, w.D), generator=gen, device=dev, dtype=torch.float32)
+    return q1.to(w.torch_dtype).contiguous()
 
 
 def shard_boundary_rows(w: Workload) -> list[tuple[int, int, int]]:

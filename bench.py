@@ -52,7 +52,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
-    ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd", "decode"],
+    ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd", "decode", "merge"],
                     help="fwd: the forward hot path (the headline line); bwd: ring_attn_bwd on the same workload; "
                          "decode: one decode step against the workload's K/V as the cache")
     return ap.parse_args()
@@ -492,6 +492,56 @@ def run_decode(args, world, rank, local):
     }))
 
 
+MERGE_METRIC = "merge of per-step partials (ring_attn_merge): HBM GB/s, 1 GPU"
+
+
+def run_merge(args, world, rank, local):
+    """Times ring_attn_merge on the workload's per-step partials: P parts of fp32 O rows
+    (B*Hq*Sq rows of one query shard's worth, D wide) and their lse, merged to bf16 O and
+    fp32 lse. Algorithmic bytes: every part read once, the result written once."""
+    from sequence_exact_attention_ring_b200 import binding, merge
+    w = synthetic.get(args.workload)
+    binding.load()
+    dev = torch.device("cuda", local if world > 1 else 0)
+    rows = w.B * w.Hq * w.Sq
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(w.seed + 900 + rank)
+    o_parts = torch.randn((w.P, rows, w.D), generator=gen, device=dev, dtype=torch.float32)
+    l_parts = torch.randn((w.P, rows), generator=gen, device=dev, dtype=torch.float32) * 4
+    nbytes = w.P * rows * (w.D + 1) * 4 + rows * (w.D * 2 + 4)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        merge(o_parts, l_parts, torch.bfloat16, stream=stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    sampler = ClockSampler(dev.index)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        merge(o_parts, l_parts, torch.bfloat16, stream=stream)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in ev), world)
+    peaks, peak_src = measured_peaks()
+    achieved = nbytes / (ms * 1e-3) / 1e9
+    clocks_all = gather_objects(clocks, world)
+    if rank != 0:
+        return
+    print(json.dumps({
+        "metric": MERGE_METRIC, "value": achieved * world, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic",
+        "config": {"workload": w.name, "parts": w.P, "rows": rows, "D": w.D, "bytes": nbytes,
+                   "l2": "parts larger than L2 (no flush)" if nbytes > 126e6 else "parts fit in L2"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                     "frac": achieved / float(peaks["hbm_gbs"]), "traffic": None,
+                     "peak_source": f"{peak_src} hbm_gbs", "kernel": "merge_kernel"},
+        "gpu_launches": args.steps,
+        "clocks": clocks_all[0] if world == 1 else {"per_rank": clocks_all},
+    }))
+
+
 def main():
     args = parse()
     world, rank, local = dist_setup(args)
@@ -502,6 +552,8 @@ def main():
             run_backward(args, world, rank, local)
         elif args.which == "decode":
             run_decode(args, world, rank, local)
+        elif args.which == "merge":
+            run_merge(args, world, rank, local)
         else:
             run_ours(args, world, rank, local)
     finally:

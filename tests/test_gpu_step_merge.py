@@ -75,6 +75,26 @@ def test_merge_kernel_against_oracle(cuda_lib, out_dtype):
     assert np.abs(lse.cpu().numpy()[fin] - L_ref[fin]).max() <= 1e-5
 
 
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("n,rows,D", [(320, 8, 128), (37, 5, 64), (1024, 3, 128)])
+def test_merge_many_parts_few_rows(cuda_lib, out_dtype, n, rows, D):
+    """The decode-shaped merge (one block per row, parts split across its threads)."""
+    g = torch.Generator().manual_seed(12 + n)
+    o = torch.randn((n, rows, D), generator=g)
+    l = torch.randn((n, rows), generator=g) * 6
+    l[::7, 0] = -torch.inf            # scattered empty parts
+    l[:, rows - 1] = -torch.inf       # an all-empty row
+    O_ref, L_ref = oracle.merge_partials(list(o.numpy()), list(l.numpy()))
+    out, lse = merge(o.cuda(), l.cuda(), out_dtype)
+    torch.cuda.synchronize()
+    tol = 1e-5 if out_dtype == torch.float32 else 2e-2
+    got = out.float().cpu().numpy()
+    assert np.abs(got - O_ref).max() <= tol
+    fin = np.isfinite(L_ref)
+    assert np.isneginf(lse.cpu().numpy()[~fin]).all() and (got[~fin] == 0).all()
+    assert np.abs(lse.cpu().numpy()[fin] - L_ref[fin]).max() <= 1e-5
+
+
 def test_watchdog_gives_up_and_context_stays_usable(cuda_lib):
     ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
     s = torch.cuda.current_stream().cuda_stream

@@ -224,9 +224,9 @@ int ring_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* out
 
 /*
  * Host only, no GPU. Walks the exact schedule and per-element masks of one pass of
- * ring_attn_bwd (pass 0: the dK/dV kernel's KV units and the query tiles each meets;
- * pass 1: the dQ kernel's query units and their backward-ring walk) with 128-row
- * tiles and adds 1 to counts[t*S + u] for every (query token t, key token u) pair
+ * ring_attn_bwd (pass 0: the dK/dV kernel's 128-key units and the 64-row query steps
+ * each meets; pass 1: the dQ kernel's 128-row query units and their backward-ring walk
+ * in 64-key steps) and adds 1 to counts[t*S + u] for every (query token t, key token u) pair
  * it lets into the gradient. counts: host S*S int32 zeroed by the caller, S <= 4096.
  * Returns the number of tile visits, or a negative error code.
  */

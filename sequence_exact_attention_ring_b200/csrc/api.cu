@@ -254,39 +254,40 @@ int64_t ring_attn_debug_bwd_visit_counts(int64_t S, int P, int causal, int layou
   int rc = check_geom(1, 1, 1, S, 128, P, causal, layout, RING_ATTN_DTYPE_BF16, &g);
   if (rc) return rc;
   if (!counts || S > 4096 || (pass != 0 && pass != 1)) return RING_ATTN_EINVAL;
-  const int T = 128;
+  const int T = 128;   // stationary tile rows (keys of the dK/dV pass, queries of the dQ pass)
+  const int TS = 64;   // rows of a streamed step
   int64_t visits = 0;
   if (pass == 0) {
-    // dK/dV pass: every KV unit, every query tile it meets, the kernel's column rule
+    // dK/dV pass: every KV unit, every query step it meets, the kernel's column rule
     for (int64_t uu = 0; uu < num_kv_units(g, T); ++uu) {
       const KvUnit U = decode_kv_unit(g, T, uu);
-      for (QWalk w = qwalk_begin(g, U, T, T); qwalk_valid(w); qwalk_next(g, w, T)) {
+      for (QWalk w = qwalk_begin(g, U, TS, T); qwalk_valid(w); qwalk_next(g, w, TS)) {
         ++visits;
         for (int r = 0; r < T; ++r) {
           const int64_t b = (int64_t)U.kt * T + r;
           if (b >= g.Sq) continue;
           const int64_t u = token_of(g, U.j, b);
-          const int cmin = bwd_first_visible_col(g, w.i, (int64_t)w.qt * T, u, T);
-          for (int c = cmin; c < T; ++c) {
-            const int64_t a = (int64_t)w.qt * T + c;
+          const int cmin = bwd_first_visible_col(g, w.i, (int64_t)w.qt * TS, u, TS);
+          for (int c = cmin; c < TS; ++c) {
+            const int64_t a = (int64_t)w.qt * TS + c;
             if (a < g.Sq) counts[token_of(g, w.i, a) * S + u] += 1;
           }
         }
       }
     }
   } else {
-    // dQ pass: every query unit, its backward-ring walk, the key limit per row
+    // dQ pass: every query unit, its backward-ring walk in key steps, the key limit per row
     for (int64_t uu = 0; uu < num_units(g, T, -1); ++uu) {
       const Unit U = decode_unit(g, T, -1, uu);
       const int64_t a0 = (int64_t)U.tb * T;
       const int64_t a_hi = (a0 + T - 1 < g.Sq - 1) ? a0 + T - 1 : g.Sq - 1;
-      for (TileWalk w = walk_begin_rev(g, U.i, a_hi, T); walk_valid(w); walk_next(g, w, a_hi, T)) {
+      for (TileWalk w = walk_begin_rev(g, U.i, a_hi, TS); walk_valid(w); walk_next(g, w, a_hi, TS)) {
         ++visits;
         for (int r = 0; r < T && a0 + r < g.Sq; ++r) {
           const int64_t a = a0 + r;
           const int64_t lim = key_limit(g, U.i, w.j, a);
-          for (int c = 0; c < T; ++c) {
-            const int64_t b = (int64_t)w.kb * T + c;
+          for (int c = 0; c < TS; ++c) {
+            const int64_t b = (int64_t)w.kb * TS + c;
             if (b < lim) counts[token_of(g, U.i, a) * S + token_of(g, w.j, b)] += 1;
           }
         }

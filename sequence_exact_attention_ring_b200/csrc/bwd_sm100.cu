@@ -16,26 +16,27 @@
 //                      a query tile's statistics are 512 contiguous bytes.
 //   bwd_dkdv_kernel    one CTA per K/V tile (b, kv head, shard j, 128 keys). As the
 //                      tile travels the backward ring it meets query shard (j - s) mod P
-//                      at step s; the CTA visits every query tile (of every query head
-//                      of the GQA group) that sees it:
+//                      at step s; the CTA visits, 64 rows at a time, every query row (of
+//                      every query head of the GQA group) that sees it:
 //                          S^T = K Q^T, dP^T = V dO^T        (SS MMAs into TMEM)
 //                          P^T, dS^T per key row              (8 warps, registers)
 //                          dV += P^T dO, dK += dS^T Q         (A operands from TMEM)
 //                      and writes dK, dV once, without atomics.
-//   bwd_dq_kernel      one CTA per query tile; it walks the K/V tiles in backward-ring
-//                      order (shard (i + s) mod P at step s):
+//   bwd_dq_kernel      one CTA per 128-row query tile; it walks the keys, 64 at a time,
+//                      in backward-ring order (shard (i + s) mod P at step s):
 //                          S = Q K^T, dP = dO V^T, then P, dS per query row,
 //                          dQ += dS K                         (A operand from TMEM)
+// Both keep two TMEM buffers of the 64-column score and dP tiles, so the tensor cores
+// compute step n + 1 (and finish step n - 1's accumulation) while the elementwise
+// warps work on step n.
 // Splitting dQ from dK/dV recomputes S and dP once more (7 instead of 5 GEMMs) and
 // in exchange needs no atomic accumulation anywhere.
 //
-// Tensor memory (512 columns) in both main kernels: the transposed or plain score
-// tile [0,128), the dP tile [128,256), accumulators from 256. Eight elementwise
-// warps split each tile: warp w owns TMEM lanes 32 (w % 4) .. +31 and columns
-// 64 (w / 4) .. +63 of the score and dP tiles; it writes its 64 bf16 P (or dS)
-// values packed into the first 32 of those columns. Each 32-column chunk is read
-// before its 16 packed columns are stored, and chunk c's packed columns overlap only
-// chunk 0's fp32 columns, so no value is overwritten before it is read.
+// Tensor memory (512 columns): score buffers [0,64) and [64,128), dP buffers [128,192)
+// and [192,256), accumulators from 256. Eight elementwise warps split each 64-column
+// tile: warp w owns TMEM lanes 32 (w % 4) .. +31 and columns 32 (w / 4) .. +31 of it;
+// it writes its 32 bf16 P (or dS) values packed into the first 16 of those columns,
+// which it has already read, so no warp overwrites a value another warp still needs.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -54,7 +55,6 @@ constexpr int BT = 128;                    // rows of every tile (keys or querie
 constexpr int BOXW = 64;                   // bf16 per TMA box row (128 bytes, 128B swizzle)
 constexpr int kBoxBytes = BT * BOXW * 2;   // 16 KiB
 constexpr int kTileBytes = BT * D * 2;     // 32 KiB
-constexpr int kStatBytes = BT * 4;         // 128 fp32 statistics of a query tile
 constexpr int kSmemLimit = 232448;
 constexpr int kThreads = 384;              // 8 elementwise warps, producer, MMA, 2 idle
 constexpr int kEwWarps = 8;
@@ -62,10 +62,7 @@ constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr uint32_t kProducerSleepNs = 64;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0;
-constexpr uint32_t kColDP = 128;
 constexpr uint32_t kColAcc = 256;
-constexpr uint32_t kIdescSS = idesc_bf16_f32(BT, BT, 0, 0);  // both operands K-major
 constexpr uint32_t kIdescTS = idesc_bf16_f32(BT, D, 0, 1);   // B MN-major (rows of the K dim)
 
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
@@ -84,8 +81,6 @@ __device__ __forceinline__ uint64_t kmajor_step(uint64_t base, int k) {
 __device__ __forceinline__ uint64_t mnmajor_step(uint64_t base, int k) {
   return base + (uint64_t)((k * 16 * 128) >> 4);
 }
-// TMEM column of K step k of a packed bf16 operand written by the two column halves.
-__device__ __forceinline__ uint32_t packed_step_col(int k) { return (uint32_t)((k / 4) * 64 + (k % 4) * 8); }
 
 // ----------------------------------------------------------------------- prep
 // One warp per padded shard-local query row (bh, i, a): lse2 = lse * log2(e) and
@@ -166,21 +161,41 @@ __device__ __forceinline__ void p_ds_chunk(const uint32_t (&s)[32], const uint32
   }
 }
 
+constexpr int TS = 64;                          // rows of a streamed step (query rows or keys)
+constexpr int kStepBoxBytes = TS * BOXW * 2;    // 8 KiB
+constexpr int kStepTileBytes = TS * D * 2;      // 16 KiB
+constexpr int kStepStatBytes = TS * 4;          // 256 B
+constexpr uint32_t kIdescSS64 = idesc_bf16_f32(BT, TS, 0, 0);  // M = 128, N = 64, both K-major
+// TMEM columns of double buffer b: the score tile (transposed in the dK/dV kernel) and the dP tile
+__device__ __forceinline__ uint32_t col_s(int b) { return (uint32_t)(64 * b); }
+__device__ __forceinline__ uint32_t col_dp(int b) { return (uint32_t)(128 + 64 * b); }
+// K step k of a 64-row K-major operand staged as two 64-column boxes of 8 KiB
+__device__ __forceinline__ uint64_t kmajor64_step(uint64_t base, int k) {
+  return base + (uint64_t)((((k / 4) * kStepBoxBytes) + (k % 4) * 32) >> 4);
+}
+// TMEM column of K step k (16 rows of the K dim) of a packed bf16 operand over 64 K
+// rows written by the two column halves (32 rows each, 16 packed columns each)
+__device__ __forceinline__ uint32_t packed64_step_col(int k) { return (uint32_t)((k / 2) * 32 + (k % 2) * 8); }
+
 // Shared memory of the dK/dV kernel: K and V tiles, then a ring of query-side slots
-// (a Q or dO tile followed by its 128 statistics).
+// (a 64-row Q or dO tile followed by its 64 statistics).
 constexpr int kA_OffK = 0;
 constexpr int kA_OffV = kTileBytes;
 constexpr int kA_OffRing = 2 * kTileBytes;
-constexpr int kA_SlotBytes = ((kTileBytes + kStatBytes + 1023) / 1024) * 1024;
-constexpr int kA_Slots = (kSmemLimit - 1024 - 64 - 512 - kA_OffRing) / kA_SlotBytes;
+constexpr int kA_SlotBytes = ((kStepTileBytes + kStepStatBytes + 1023) / 1024) * 1024;
+constexpr int kA_SlotsFit = (kSmemLimit - 1024 - 64 - 512 - kA_OffRing) / kA_SlotBytes;
+constexpr int kA_Slots = kA_SlotsFit < 8 ? kA_SlotsFit : 8;
 constexpr int kA_OffBar = kA_OffRing + kA_Slots * kA_SlotBytes;
-enum BarA { kA_KVFull = 0, kA_STFull = 1, kA_PReady = 2, kA_Done = 3, kA_Drain = 4, kA_Ring = 5 };
+enum BarA { kA_KVFull = 0, kA_STFull = 1, kA_PReady = 3, kA_Done = 5, kA_Drain = 6, kA_Ring = 7 };
 constexpr int kA_NumBars = kA_Ring + 2 * kA_Slots;
 constexpr int kA_OffMisc = kA_OffBar + kA_NumBars * 8;
 constexpr int kA_SmemBytes = kA_OffMisc + 64 + 1024;
-static_assert(kA_Slots >= 2, "need a Q and a dO slot");
+static_assert(kA_Slots >= 4, "need two steps of Q and dO slots");
 static_assert(kA_SmemBytes <= kSmemLimit, "shared memory budget");
 
+// dK/dV: one CTA per 128-key tile; query rows arrive in steps of 64. TMEM holds two
+// buffers of (S^T 64 columns, dP^T 64 columns) and the dV, dK accumulators, so the
+// products of step n + 1 run while the elementwise warps work on step n.
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -198,8 +213,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&bars[kA_KVFull], 1);
-    mbar_init(&bars[kA_STFull], 1);
-    mbar_init(&bars[kA_PReady], kEwWarps);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars[kA_STFull + b], 1);
+      mbar_init(&bars[kA_PReady + b], kEwWarps);
+    }
     mbar_init(&bars[kA_Done], 1);
     mbar_init(&bars[kA_Drain], 1);
     for (int s = 0; s < 2 * kA_Slots; ++s) mbar_init(&bars[kA_Ring + s], 1);
@@ -218,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const KvUnit U = decode_kv_unit(g, BT, blockIdx.x);
   const int bh_kv = U.b * g.Hkv + U.g;
   const int rep = g.Hq / g.Hkv;
-  const int64_t N = qwalk_count(g, U, BT, BT);  // query tiles met (x2 loads each)
+  const int64_t N = qwalk_count(g, U, TS, BT);  // query steps met (x2 loads each)
   auto slot_of = [&](int64_t m) { return (int)(m % kA_Slots); };
   auto phase_of = [&](int64_t m) { return (uint32_t)((m / kA_Slots) & 1); };
 
@@ -236,19 +253,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       int64_t m = 0;
       bool ok = true;
-      for (QWalk w = qwalk_begin(g, U, BT, BT); qwalk_valid(w) && ok; qwalk_next(g, w, BT)) {
+      for (QWalk w = qwalk_begin(g, U, TS, BT); qwalk_valid(w) && ok; qwalk_next(g, w, TS)) {
         const int bh_q = U.b * g.Hq + U.g * rep + w.hr;
-        const int64_t a0 = (int64_t)w.qt * BT;
+        const int64_t a0 = (int64_t)w.qt * TS;
         shard_map_coords(g, w.i, a0, c1, c2);
         const int64_t stat = ((int64_t)bh_q * g.P + w.i) * p.sq_pad + a0;
         for (int kind = 0; kind < 2; ++kind, ++m) {
           const int slot = slot_of(m);
           if (!(ok = mbar_wait_backoff<false>(&empty[slot], phase_of(m) ^ 1, wd, kProducerSleepNs))) break;
           uint8_t* dst = smem + kA_OffRing + slot * kA_SlotBytes;
-          mbar_arrive_expect_tx(&full[slot], kTileBytes + kStatBytes);
+          mbar_arrive_expect_tx(&full[slot], kStepTileBytes + kStepStatBytes);
           const CUtensorMap* tm = kind == 0 ? &tm_q : &tm_do;
-          for (int bx = 0; bx < 2; ++bx) tma_load_4d(dst + bx * kBoxBytes, tm, &full[slot], bx * BOXW, c1, c2, bh_q);
-          bulk_load(dst + kTileBytes, (kind == 0 ? p.lse2 : p.delta) + stat, kStatBytes, &full[slot]);
+          for (int bx = 0; bx < 2; ++bx)
+            tma_load_4d(dst + bx * kStepBoxBytes, tm, &full[slot], bx * BOXW, c1, c2, bh_q);
+          bulk_load(dst + kStepTileBytes, (kind == 0 ? p.lse2 : p.delta) + stat, kStepStatBytes, &full[slot]);
         }
       }
       if (!ok) {
@@ -265,37 +283,47 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t dK = smem_desc_sw128(sbase + kA_OffK, 0, 1024);
     const uint64_t dV = smem_desc_sw128(sbase + kA_OffV, 0, 1024);
     auto all = [&](bool r) { return __all_sync(0xffffffffu, r); };
+    auto slot_addr = [&](int64_t m) { return sbase + kA_OffRing + slot_of(m) * kA_SlotBytes; };
+    // S^T = K Q^T and dP^T = V dO^T of step n into buffer n % 2
+    auto issue_st = [&](int64_t n) -> bool {
+      if (!all(mbar_wait(&full[slot_of(2 * n)], phase_of(2 * n), wd))) return false;
+      if (!all(mbar_wait(&full[slot_of(2 * n + 1)], phase_of(2 * n + 1), wd))) return false;
+      tc_fence_after();
+      const int b = (int)(n & 1);
+      const uint64_t bq = smem_desc_sw128(slot_addr(2 * n), 0, 1024);
+      const uint64_t bd = smem_desc_sw128(slot_addr(2 * n + 1), 0, 1024);
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k)
+        if (issuer) mma_ss(tmem + col_s(b), kmajor_step(dK, k), kmajor64_step(bq, k), kIdescSS64, k > 0);
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k)
+        if (issuer) mma_ss(tmem + col_dp(b), kmajor_step(dV, k), kmajor64_step(bd, k), kIdescSS64, k > 0);
+      if (issuer) mma_commit(&bars[kA_STFull + b]);
+      return true;
+    };
     bool ok = N > 0 && all(mbar_wait(&bars[kA_KVFull], 0, wd));
+    if (ok) ok = issue_st(0);
+    if (ok && N > 1) ok = issue_st(1);
     for (int64_t n = 0; ok && n < N; ++n) {
-      const int sq = slot_of(2 * n), sd = slot_of(2 * n + 1);
-      const uint32_t aq = sbase + kA_OffRing + sq * kA_SlotBytes;
-      const uint32_t ad = sbase + kA_OffRing + sd * kA_SlotBytes;
-      if (!(ok = all(mbar_wait(&full[sq], phase_of(2 * n), wd)))) break;
-      if (!(ok = all(mbar_wait(&full[sd], phase_of(2 * n + 1), wd)))) break;
+      const int b = (int)(n & 1);
+      if (!(ok = all(mbar_wait(&bars[kA_PReady + b], (uint32_t)((n >> 1) & 1), wd)))) break;
       tc_fence_after();
-      const uint64_t bq = smem_desc_sw128(aq, 0, 1024), bd = smem_desc_sw128(ad, 0, 1024);
+      const uint64_t mq = smem_desc_sw128(slot_addr(2 * n), kStepBoxBytes, 1024);
+      const uint64_t md = smem_desc_sw128(slot_addr(2 * n + 1), kStepBoxBytes, 1024);
 #pragma unroll
-      for (int k = 0; k < D / 16; ++k)
-        if (issuer) mma_ss(tmem + kColS, kmajor_step(dK, k), kmajor_step(bq, k), kIdescSS, k > 0);
-#pragma unroll
-      for (int k = 0; k < D / 16; ++k)
-        if (issuer) mma_ss(tmem + kColDP, kmajor_step(dV, k), kmajor_step(bd, k), kIdescSS, k > 0);
-      if (issuer) mma_commit(&bars[kA_STFull]);
-      if (!(ok = all(mbar_wait(&bars[kA_PReady], (uint32_t)(n & 1), wd)))) break;
-      tc_fence_after();
-      const uint64_t mq = smem_desc_sw128(aq, kBoxBytes, 1024), md = smem_desc_sw128(ad, kBoxBytes, 1024);
-#pragma unroll
-      for (int k = 0; k < BT / 16; ++k)  // dV += P^T dO
-        if (issuer) mma_ts(tmem + kColAcc, tmem + kColS + packed_step_col(k), mnmajor_step(md, k), kIdescTS,
+      for (int k = 0; k < TS / 16; ++k)  // dV += P^T dO
+        if (issuer) mma_ts(tmem + kColAcc, tmem + col_s(b) + packed64_step_col(k), mnmajor_step(md, k), kIdescTS,
                            !(n == 0 && k == 0));
 #pragma unroll
-      for (int k = 0; k < BT / 16; ++k)  // dK += dS^T Q
-        if (issuer) mma_ts(tmem + kColAcc + D, tmem + kColDP + packed_step_col(k), mnmajor_step(mq, k), kIdescTS,
+      for (int k = 0; k < TS / 16; ++k)  // dK += dS^T Q
+        if (issuer) mma_ts(tmem + kColAcc + D, tmem + col_dp(b) + packed64_step_col(k), mnmajor_step(mq, k), kIdescTS,
                            !(n == 0 && k == 0));
       if (issuer) {
-        mma_commit(&empty[sq]);
-        mma_commit(&empty[sd]);
+        mma_commit(&empty[slot_of(2 * n)]);
+        mma_commit(&empty[slot_of(2 * n + 1)]);
       }
+      // buffer b is free for step n + 2 once these products have read its P and dS
+      if (n + 2 < N && !(ok = issue_st(n + 2))) break;
     }
     if (issuer) {
       mma_commit(&bars[kA_Done]);
@@ -304,51 +332,49 @@ __global__ void __launch_bounds__(kThreads, 1)
     drain_wait(&bars[kA_Drain], 0, p.watchdog_ns);
   } else if (warp < kEwWarps) {
     // ------------------------------------------------------------- elementwise + epilogue
+    // warp = 4 hh + wq: TMEM lanes 32 wq (key rows), query columns 32 hh .. 32 hh + 31 of a step
     const int wq = warp % 4, hh = warp / 4;
     const int r = wq * 32 + lane;
-    const int64_t b = (int64_t)U.kt * BT + r;  // key row of shard j
-    const int64_t u = token_of(g, U.j, b);
+    const int64_t bk = (int64_t)U.kt * BT + r;  // key row of shard j
+    const int64_t u = token_of(g, U.j, bk);
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-    const uint32_t tS = tmem + lane_off + kColS + hh * 64;
-    const uint32_t tDP = tmem + lane_off + kColDP + hh * 64;
     int64_t n = 0;
     bool ok = true;
-    int row_i = -1;       // query shard of the cached first visible row
-    int64_t row0 = 0;     // first row of shard row_i whose token is >= u
-    for (QWalk w = qwalk_begin(g, U, BT, BT); qwalk_valid(w); qwalk_next(g, w, BT), ++n) {
+    int row_i = -1;    // query shard of the cached first visible row
+    int64_t row0 = 0;  // first row of shard row_i whose token is >= u
+    for (QWalk w = qwalk_begin(g, U, TS, BT); qwalk_valid(w); qwalk_next(g, w, TS), ++n) {
+      const int b = (int)(n & 1);
       const int sq = slot_of(2 * n), sd = slot_of(2 * n + 1);
-      if (!(ok = mbar_wait(&bars[kA_STFull], (uint32_t)(n & 1), wd))) break;
+      if (!(ok = mbar_wait(&bars[kA_STFull + b], (uint32_t)((n >> 1) & 1), wd))) break;
       // the statistics came with the tiles: wait on their barriers too (already complete)
       if (!(ok = mbar_wait(&full[sq], phase_of(2 * n), wd) && mbar_wait(&full[sd], phase_of(2 * n + 1), wd))) break;
       tc_fence_after();
-      const float* lse2c = reinterpret_cast<const float*>(smem + kA_OffRing + sq * kA_SlotBytes + kTileBytes);
-      const float* deltac = reinterpret_cast<const float*>(smem + kA_OffRing + sd * kA_SlotBytes + kTileBytes);
+      const float* lse2c = reinterpret_cast<const float*>(smem + kA_OffRing + sq * kA_SlotBytes + kStepTileBytes);
+      const float* deltac = reinterpret_cast<const float*>(smem + kA_OffRing + sd * kA_SlotBytes + kStepTileBytes);
       if (w.i != row_i) {
         row_i = w.i;
         row0 = g.causal ? first_row_at_or_after(g, w.i, u) : 0;
       }
-      const int64_t cm = row0 - (int64_t)w.qt * BT;
-      const int cmin = cm < 0 ? 0 : (cm > BT ? BT : (int)cm);
-#pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        uint32_t s[32], dp[32], pp[16], pds[16];
-        tmem_ld32(tS + cc * 32, s);
-        tmem_ld32(tDP + cc * 32, dp);
-        tmem_wait_ld();
-        const int c0 = hh * 64 + cc * 32;
-        p_ds_chunk(s, dp, lse2c + c0, deltac + c0, 0.f, 0.f, true, p.scale_log2, c0, cmin, BT, pp, pds);
-        tmem_st16(tS + cc * 16, pp);
-        tmem_st16(tDP + cc * 16, pds);
-      }
+      const int64_t cm = row0 - (int64_t)w.qt * TS;
+      const int cmin = cm < 0 ? 0 : (cm > TS ? TS : (int)cm);
+      uint32_t sv[32], dpv[32], pp[16], pds[16];
+      tmem_ld32(tmem + lane_off + col_s(b) + 32 * hh, sv);
+      tmem_ld32(tmem + lane_off + col_dp(b) + 32 * hh, dpv);
+      tmem_wait_ld();
+      p_ds_chunk(sv, dpv, lse2c + 32 * hh, deltac + 32 * hh, 0.f, 0.f, true, p.scale_log2, 32 * hh, cmin, TS, pp,
+                 pds);
+      // the packed columns overlap only this warp's own, already loaded fp32 columns
+      tmem_st16(tmem + lane_off + col_s(b) + 32 * hh, pp);
+      tmem_st16(tmem + lane_off + col_dp(b) + 32 * hh, pds);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[kA_PReady]);
+      if (lane == 0) mbar_arrive(&bars[kA_PReady + b]);
     }
     const bool have = n > 0 && ok && mbar_wait(&bars[kA_Done], 0, wd);
     if (have || n == 0) {
       tc_fence_after();
-      const bool row_ok = b < g.Sq;
+      const bool row_ok = bk < g.Sq;
       const int64_t out_row = (int64_t)bh_kv * g.S + (row_ok ? u : 0);
       const uint32_t tAcc = tmem + lane_off + kColAcc + hh * 64;
       store_row_cols<64>(tAcc, n > 0, row_ok, 1.f, false, p.out1, out_row, D, hh * 64);         // dV
@@ -364,19 +390,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Shared memory of the dQ kernel: Q and dO once, then a ring of K/V tile slots.
+// Shared memory of the dQ kernel: Q and dO once, then a ring of 64-key K or V slots.
 constexpr int kB_OffQ = 0;
 constexpr int kB_OffDO = kTileBytes;
 constexpr int kB_OffRing = 2 * kTileBytes;
-constexpr int kB_Slots = (kSmemLimit - 1024 - 64 - 512 - kB_OffRing) / kTileBytes;
-constexpr int kB_OffBar = kB_OffRing + kB_Slots * kTileBytes;
-enum BarB { kB_QFull = 0, kB_SFull = 1, kB_PReady = 2, kB_Done = 3, kB_Drain = 4, kB_Ring = 5 };
+constexpr int kB_SlotsFit = (kSmemLimit - 1024 - 64 - 512 - kB_OffRing) / kStepTileBytes;
+constexpr int kB_Slots = kB_SlotsFit < 10 ? kB_SlotsFit : 10;
+constexpr int kB_OffBar = kB_OffRing + kB_Slots * kStepTileBytes;
+enum BarB { kB_QFull = 0, kB_SFull = 1, kB_PReady = 3, kB_Done = 5, kB_Drain = 6, kB_Ring = 7 };
 constexpr int kB_NumBars = kB_Ring + 2 * kB_Slots;
 constexpr int kB_OffMisc = kB_OffBar + kB_NumBars * 8;
 constexpr int kB_SmemBytes = kB_OffMisc + 64 + 1024;
-static_assert(kB_Slots >= 2, "need a K and a V slot");
+static_assert(kB_Slots >= 4, "need two steps of K and V slots");
 static_assert(kB_SmemBytes <= kSmemLimit, "shared memory budget");
 
+// dQ: one CTA per 128-row query tile; keys arrive in steps of 64 along the backward
+// ring. TMEM holds two buffers of (S 64 columns, dP 64 columns) and the dQ accumulator.
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -394,8 +423,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&bars[kB_QFull], 1);
-    mbar_init(&bars[kB_SFull], 1);
-    mbar_init(&bars[kB_PReady], kEwWarps);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars[kB_SFull + b], 1);
+      mbar_init(&bars[kB_PReady + b], kEwWarps);
+    }
     mbar_init(&bars[kB_Done], 1);
     mbar_init(&bars[kB_Drain], 1);
     for (int s = 0; s < 2 * kB_Slots; ++s) mbar_init(&bars[kB_Ring + s], 1);
@@ -416,7 +447,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t a_hi = (a0 + BT - 1 < g.Sq - 1) ? a0 + BT - 1 : g.Sq - 1;
   const int bh_q = U.b * g.Hq + U.h;
   const int bh_kv = U.b * g.Hkv + U.h / (g.Hq / g.Hkv);
-  const int64_t N = unit_tile_count(g, U.i, a_hi, BT, 0, g.P);  // the same tiles in either ring direction
+  const int64_t N = unit_tile_count(g, U.i, a_hi, TS, 0, g.P);  // the same steps in either ring direction
   auto slot_of = [&](int64_t m) { return (int)(m % kB_Slots); };
   auto phase_of = [&](int64_t m) { return (uint32_t)((m / kB_Slots) & 1); };
 
@@ -434,16 +465,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       int64_t m = 0;
       bool ok = true;
-      for (TileWalk w = walk_begin_rev(g, U.i, a_hi, BT); walk_valid(w) && ok; walk_next(g, w, a_hi, BT)) {
-        shard_map_coords(g, w.j, (int64_t)w.kb * BT, c1, c2);
+      for (TileWalk w = walk_begin_rev(g, U.i, a_hi, TS); walk_valid(w) && ok; walk_next(g, w, a_hi, TS)) {
+        shard_map_coords(g, w.j, (int64_t)w.kb * TS, c1, c2);
         for (int kind = 0; kind < 2; ++kind, ++m) {
           const int slot = slot_of(m);
           if (!(ok = mbar_wait_backoff<false>(&empty[slot], phase_of(m) ^ 1, wd, kProducerSleepNs))) break;
-          uint8_t* dst = smem + kB_OffRing + slot * kTileBytes;
-          mbar_arrive_expect_tx(&full[slot], kTileBytes);
+          uint8_t* dst = smem + kB_OffRing + slot * kStepTileBytes;
+          mbar_arrive_expect_tx(&full[slot], kStepTileBytes);
           const CUtensorMap* tm = kind == 0 ? &tm_k : &tm_v;
           for (int bx = 0; bx < 2; ++bx)
-            tma_load_4d(dst + bx * kBoxBytes, tm, &full[slot], bx * BOXW, c1, c2, bh_kv);
+            tma_load_4d(dst + bx * kStepBoxBytes, tm, &full[slot], bx * BOXW, c1, c2, bh_kv);
         }
       }
       if (!ok) {
@@ -459,33 +490,41 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t dQd = smem_desc_sw128(sbase + kB_OffQ, 0, 1024);
     const uint64_t dOd = smem_desc_sw128(sbase + kB_OffDO, 0, 1024);
     auto all = [&](bool r) { return __all_sync(0xffffffffu, r); };
-    bool ok = N > 0 && all(mbar_wait(&bars[kB_QFull], 0, wd));
-    for (int64_t n = 0; ok && n < N; ++n) {
-      const int sk = slot_of(2 * n), sv = slot_of(2 * n + 1);
-      const uint32_t ak = sbase + kB_OffRing + sk * kTileBytes;
-      const uint32_t av = sbase + kB_OffRing + sv * kTileBytes;
-      if (!(ok = all(mbar_wait(&full[sk], phase_of(2 * n), wd)))) break;
-      if (!(ok = all(mbar_wait(&full[sv], phase_of(2 * n + 1), wd)))) break;
+    auto slot_addr = [&](int64_t m) { return sbase + kB_OffRing + slot_of(m) * kStepTileBytes; };
+    // S = Q K^T and dP = dO V^T of step n into buffer n % 2
+    auto issue_sd = [&](int64_t n) -> bool {
+      if (!all(mbar_wait(&full[slot_of(2 * n)], phase_of(2 * n), wd))) return false;
+      if (!all(mbar_wait(&full[slot_of(2 * n + 1)], phase_of(2 * n + 1), wd))) return false;
       tc_fence_after();
-      const uint64_t bk = smem_desc_sw128(ak, 0, 1024), bv = smem_desc_sw128(av, 0, 1024);
+      const int b = (int)(n & 1);
+      const uint64_t bk = smem_desc_sw128(slot_addr(2 * n), 0, 1024);
+      const uint64_t bv = smem_desc_sw128(slot_addr(2 * n + 1), 0, 1024);
 #pragma unroll
-      for (int k = 0; k < D / 16; ++k)  // S = Q K^T
-        if (issuer) mma_ss(tmem + kColS, kmajor_step(dQd, k), kmajor_step(bk, k), kIdescSS, k > 0);
+      for (int k = 0; k < D / 16; ++k)
+        if (issuer) mma_ss(tmem + col_s(b), kmajor_step(dQd, k), kmajor64_step(bk, k), kIdescSS64, k > 0);
 #pragma unroll
-      for (int k = 0; k < D / 16; ++k)  // dP = dO V^T
-        if (issuer) mma_ss(tmem + kColDP, kmajor_step(dOd, k), kmajor_step(bv, k), kIdescSS, k > 0);
+      for (int k = 0; k < D / 16; ++k)
+        if (issuer) mma_ss(tmem + col_dp(b), kmajor_step(dOd, k), kmajor64_step(bv, k), kIdescSS64, k > 0);
       if (issuer) {
-        mma_commit(&bars[kB_SFull]);
-        mma_commit(&empty[sv]);  // V is no longer needed once dP is done
+        mma_commit(&bars[kB_SFull + b]);
+        mma_commit(&empty[slot_of(2 * n + 1)]);  // V is no longer needed once dP is done
       }
-      if (!(ok = all(mbar_wait(&bars[kB_PReady], (uint32_t)(n & 1), wd)))) break;
+      return true;
+    };
+    bool ok = N > 0 && all(mbar_wait(&bars[kB_QFull], 0, wd));
+    if (ok) ok = issue_sd(0);
+    if (ok && N > 1) ok = issue_sd(1);
+    for (int64_t n = 0; ok && n < N; ++n) {
+      const int b = (int)(n & 1);
+      if (!(ok = all(mbar_wait(&bars[kB_PReady + b], (uint32_t)((n >> 1) & 1), wd)))) break;
       tc_fence_after();
-      const uint64_t mk = smem_desc_sw128(ak, kBoxBytes, 1024);
+      const uint64_t mk = smem_desc_sw128(slot_addr(2 * n), kStepBoxBytes, 1024);
 #pragma unroll
-      for (int k = 0; k < BT / 16; ++k)  // dQ += dS K
-        if (issuer) mma_ts(tmem + kColAcc, tmem + kColS + packed_step_col(k), mnmajor_step(mk, k), kIdescTS,
+      for (int k = 0; k < TS / 16; ++k)  // dQ += dS K
+        if (issuer) mma_ts(tmem + kColAcc, tmem + col_s(b) + packed64_step_col(k), mnmajor_step(mk, k), kIdescTS,
                            !(n == 0 && k == 0));
-      if (issuer) mma_commit(&empty[sk]);
+      if (issuer) mma_commit(&empty[slot_of(2 * n)]);
+      if (n + 2 < N && !(ok = issue_sd(n + 2))) break;
     }
     if (issuer) {
       mma_commit(&bars[kB_Done]);
@@ -494,6 +533,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     drain_wait(&bars[kB_Drain], 0, p.watchdog_ns);
   } else if (warp < kEwWarps) {
     // ------------------------------------------------------------- elementwise + epilogue
+    // warp = 4 hh + wq: TMEM lanes 32 wq (query rows), keys 32 hh .. 32 hh + 31 of a step
     const int wq = warp % 4, hh = warp / 4;
     const int r = wq * 32 + lane;
     const int64_t a = a0 + r;
@@ -501,28 +541,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float row_lse2 = p.lse2[stat];
     const float row_delta = p.delta[stat];
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-    const uint32_t tS = tmem + lane_off + kColS + hh * 64;
-    const uint32_t tDP = tmem + lane_off + kColDP + hh * 64;
     int64_t n = 0;
     bool ok = true;
-    for (TileWalk w = walk_begin_rev(g, U.i, a_hi, BT); walk_valid(w); walk_next(g, w, a_hi, BT), ++n) {
-      if (!(ok = mbar_wait(&bars[kB_SFull], (uint32_t)(n & 1), wd))) break;
+    for (TileWalk w = walk_begin_rev(g, U.i, a_hi, TS); walk_valid(w); walk_next(g, w, a_hi, TS), ++n) {
+      const int b = (int)(n & 1);
+      if (!(ok = mbar_wait(&bars[kB_SFull + b], (uint32_t)((n >> 1) & 1), wd))) break;
       tc_fence_after();
-      const int cut = visible_keys<BT>((int64_t)w.kb * BT, key_limit(g, U.i, w.j, a));
-#pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        uint32_t s[32], dp[32], pp[16], pds[16];
-        tmem_ld32(tS + cc * 32, s);
-        tmem_ld32(tDP + cc * 32, dp);
-        tmem_wait_ld();
-        const int c0 = hh * 64 + cc * 32;
-        p_ds_chunk(s, dp, nullptr, nullptr, row_lse2, row_delta, false, p.scale_log2, c0, 0, cut, pp, pds);
-        tmem_st16(tS + cc * 16, pds);  // only dS feeds the dQ MMA
-      }
+      const int cut = visible_keys<TS>((int64_t)w.kb * TS, key_limit(g, U.i, w.j, a));
+      uint32_t sv[32], dpv[32], pp[16], pds[16];
+      tmem_ld32(tmem + lane_off + col_s(b) + 32 * hh, sv);
+      tmem_ld32(tmem + lane_off + col_dp(b) + 32 * hh, dpv);
+      tmem_wait_ld();
+      p_ds_chunk(sv, dpv, nullptr, nullptr, row_lse2, row_delta, false, p.scale_log2, 32 * hh, 0, cut, pp, pds);
+      tmem_st16(tmem + lane_off + col_s(b) + 32 * hh, pds);  // only dS feeds the dQ MMA
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[kB_PReady]);
+      if (lane == 0) mbar_arrive(&bars[kB_PReady + b]);
     }
     const bool have = n > 0 && ok && mbar_wait(&bars[kB_Done], 0, wd);
     if (have || n == 0) {
@@ -561,12 +596,17 @@ int launch_bwd_sm100(const void* q, const void* k, const void* v, const void* ou
                                                               static_cast<const uint16_t*>(dout), lse, lse2, delta,
                                                               g, sq_pad, rows);
   if (cudaGetLastError() != cudaSuccess) return RING_ATTN_ECUDA;
-  CUtensorMap mq, mdo, mk, mv;
+  // 128-row boxes for the stationary tiles, 64-row boxes for the streamed steps
+  CUtensorMap mq, mdo, mk, mv, mq64, mdo64, mk64, mv64;
   int rc;
   if ((rc = encode_shard_map(&mq, q, g, g.Hq, D, BT)) != 0) return rc;
   if ((rc = encode_shard_map(&mdo, dout, g, g.Hq, D, BT)) != 0) return rc;
   if ((rc = encode_shard_map(&mk, k, g, g.Hkv, D, BT)) != 0) return rc;
   if ((rc = encode_shard_map(&mv, v, g, g.Hkv, D, BT)) != 0) return rc;
+  if ((rc = encode_shard_map(&mq64, q, g, g.Hq, D, TS)) != 0) return rc;
+  if ((rc = encode_shard_map(&mdo64, dout, g, g.Hq, D, TS)) != 0) return rc;
+  if ((rc = encode_shard_map(&mk64, k, g, g.Hkv, D, TS)) != 0) return rc;
+  if ((rc = encode_shard_map(&mv64, v, g, g.Hkv, D, TS)) != 0) return rc;
   Params p;
   p.g = g;
   p.lse2 = lse2;
@@ -585,11 +625,11 @@ int launch_bwd_sm100(const void* q, const void* k, const void* v, const void* ou
   if (kv_units > 0x7fffffff || q_units > 0x7fffffff) return RING_ATTN_EINVAL;
   p.out0 = dk;
   p.out1 = dv;
-  bwd_dkdv_kernel<<<(unsigned)kv_units, kThreads, kA_SmemBytes, stream>>>(mq, mdo, mk, mv, p);
+  bwd_dkdv_kernel<<<(unsigned)kv_units, kThreads, kA_SmemBytes, stream>>>(mq64, mdo64, mk, mv, p);
   if (cudaGetLastError() != cudaSuccess) return RING_ATTN_ECUDA;
   p.out0 = dq;
   p.out1 = nullptr;
-  bwd_dq_kernel<<<(unsigned)q_units, kThreads, kB_SmemBytes, stream>>>(mq, mdo, mk, mv, p);
+  bwd_dq_kernel<<<(unsigned)q_units, kThreads, kB_SmemBytes, stream>>>(mq, mdo, mk64, mv64, p);
   return cudaGetLastError() == cudaSuccess ? RING_ATTN_OK : RING_ATTN_ECUDA;
 }
 

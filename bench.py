@@ -317,24 +317,27 @@ def run_ours(args, world, rank, local):
     # ---- end to end: pinned host buffers, H2D + kernel + D2H inside the timed region
     e2e = None
     if not args.no_e2e:
+        # Host-resident inputs through the public HostRunner: every step copies its q, k, v
+        # in from pinned memory and its out, lse back; two device buffer sets and a copy
+        # stream let one step's copies overlap another step's kernel.
         qh, kh, vh = q.cpu().pin_memory(), k.cpu().pin_memory(), v.cpu().pin_memory()
-        runner = HostRunner(q.shape, k.shape, q.dtype, w.P, w.causal, w.layout, w.scale, device=dev)
-        runner.run(qh, kh, vh, stream)
-        torch.cuda.synchronize(dev)
         del out
+        runner = HostRunner(q.shape, k.shape, q.dtype, w.P, w.causal, w.layout, w.scale, device=dev, buffers=2)
+        copy_stream = torch.cuda.Stream(dev)
+        runner.run_steps([(qh, kh, vh)], copy_stream, stream)
+        torch.cuda.synchronize(dev)
         barrier(world)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
-        e_steps = max(1, min(args.steps, 3))
-        e0.record(stream)
-        for _ in range(e_steps):
-            runner.run(qh, kh, vh, stream)
-        e1.record(stream)
+        e_steps = max(2, min(args.steps, 4))
+        e0.record(copy_stream)
+        runner.run_steps([(qh, kh, vh)] * e_steps, copy_stream, stream)
+        e1.record(copy_stream)
         torch.cuda.synchronize(dev)
         e_ms = max_over_ranks(e0.elapsed_time(e1), world)
         e2e = {"value": flops * world * e_steps / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": runner.h2d_bytes() * world, "d2h_bytes_per_step": runner.d2h_bytes() * world,
-               "steps": e_steps}
+               "steps": e_steps, "pipelined": "2 device buffer sets, copies on their own stream"}
 
     clocks_all = gather_objects(clocks, world)
     statuses = gather_objects(st, world)

@@ -173,23 +173,36 @@ def status(workspace: torch.Tensor, stream=None) -> int:
 
 class HostRunner:
     """End-to-end path for host-resident inputs: pinned host -> device copies,
-    ring_attn_fwd, device -> pinned host copies, all on one stream.
+    ring_attn_fwd, device -> pinned host copies.
 
-    Device buffers are allocated once (by torch) and reused across calls.
+    Device buffers are allocated once (by torch) and reused across calls. `run` does
+    one step on one stream. `run_steps` runs many steps as a pipeline over `buffers`
+    device buffer sets and two streams: the copies of one step overlap the kernel of
+    another, as a serving loop would run them.
     """
 
-    def __init__(self, shape_q, shape_kv, dtype, P, causal=True, layout="striped", scale=None, device="cuda"):
+    def __init__(self, shape_q, shape_kv, dtype, P, causal=True, layout="striped", scale=None, device="cuda",
+                 buffers=1):
         self.P, self.causal, self.layout = P, causal, layout
         B, Hq, S, D = shape_q
         self.scale = 1.0 / math.sqrt(D) if scale is None else scale
-        self.q = torch.empty(shape_q, dtype=dtype, device=device)
-        self.k = torch.empty(shape_kv, dtype=dtype, device=device)
-        self.v = torch.empty(shape_kv, dtype=dtype, device=device)
-        self.out = torch.empty(shape_q, dtype=dtype, device=device)
-        self.lse = torch.empty((B, Hq, S), dtype=torch.float32, device=device)
-        self.out_host = torch.empty(shape_q, dtype=dtype, pin_memory=True)
-        self.lse_host = torch.empty((B, Hq, S), dtype=torch.float32, pin_memory=True)
-        self.ws = torch.empty(workspace_bytes(self.q, self.k, P, causal, layout), dtype=torch.uint8, device=device)
+        self.sets = []
+        for _ in range(max(1, buffers)):
+            st = {
+                "q": torch.empty(shape_q, dtype=dtype, device=device),
+                "k": torch.empty(shape_kv, dtype=dtype, device=device),
+                "v": torch.empty(shape_kv, dtype=dtype, device=device),
+                "out": torch.empty(shape_q, dtype=dtype, device=device),
+                "lse": torch.empty((B, Hq, S), dtype=torch.float32, device=device),
+                "out_host": torch.empty(shape_q, dtype=dtype, pin_memory=True),
+                "lse_host": torch.empty((B, Hq, S), dtype=torch.float32, pin_memory=True),
+            }
+            st["ws"] = torch.empty(workspace_bytes(st["q"], st["k"], P, causal, layout), dtype=torch.uint8,
+                                   device=device)
+            self.sets.append(st)
+        first = self.sets[0]
+        self.q, self.k, self.v, self.out, self.lse = first["q"], first["k"], first["v"], first["out"], first["lse"]
+        self.out_host, self.lse_host, self.ws = first["out_host"], first["lse_host"], first["ws"]
 
     def h2d_bytes(self) -> int:
         return sum(t.numel() * t.element_size() for t in (self.q, self.k, self.v))
@@ -197,14 +210,59 @@ class HostRunner:
     def d2h_bytes(self) -> int:
         return self.out.numel() * self.out.element_size() + self.lse.numel() * 4
 
+    def _forward(self, st, stream):
+        ring_attention(st["q"], st["k"], st["v"], self.P, self.causal, self.layout, self.scale, out=st["out"],
+                       lse=st["lse"], workspace=st["ws"], stream=stream)
+
     def run(self, q_host, k_host, v_host, stream=None):
         s = stream if stream is not None else torch.cuda.current_stream()
+        st = self.sets[0]
         with torch.cuda.stream(s):
-            self.q.copy_(q_host, non_blocking=True)
-            self.k.copy_(k_host, non_blocking=True)
-            self.v.copy_(v_host, non_blocking=True)
-            ring_attention(self.q, self.k, self.v, self.P, self.causal, self.layout, self.scale, out=self.out,
-                           lse=self.lse, workspace=self.ws, stream=s)
-            self.out_host.copy_(self.out, non_blocking=True)
-            self.lse_host.copy_(self.lse, non_blocking=True)
-        return self.out_host, self.lse_host
+            st["q"].copy_(q_host, non_blocking=True)
+            st["k"].copy_(k_host, non_blocking=True)
+            st["v"].copy_(v_host, non_blocking=True)
+            self._forward(st, s)
+            st["out_host"].copy_(st["out"], non_blocking=True)
+            st["lse_host"].copy_(st["lse"], non_blocking=True)
+        return st["out_host"], st["lse_host"]
+
+    def run_steps(self, batches, copy_stream, compute_stream):
+        """Pipelined steps over the buffer sets: every (q_host, k_host, v_host) in `batches`
+        is copied in on `copy_stream`, folded on `compute_stream` once its copy landed,
+        and its out and lse copied back on `copy_stream` once the kernel finished. Step n
+        uses set n % buffers; its host results stay valid until step n + buffers starts.
+        Asynchronous: synchronize copy_stream to wait for everything."""
+        nb = len(self.sets)
+        batches = list(batches)
+        h2d_done = [torch.cuda.Event() for _ in batches]
+        fwd_done = [torch.cuda.Event() for _ in batches]
+
+        def h2d(n):
+            st = self.sets[n % nb]
+            qh, kh, vh = batches[n]
+            with torch.cuda.stream(copy_stream):
+                st["q"].copy_(qh, non_blocking=True)
+                st["k"].copy_(kh, non_blocking=True)
+                st["v"].copy_(vh, non_blocking=True)
+                h2d_done[n].record(copy_stream)
+
+        def d2h(n):
+            st = self.sets[n % nb]
+            copy_stream.wait_event(fwd_done[n])
+            with torch.cuda.stream(copy_stream):
+                st["out_host"].copy_(st["out"], non_blocking=True)
+                st["lse_host"].copy_(st["lse"], non_blocking=True)
+
+        # copy stream order: H2D of the first `nb` steps, then for each step its D2H
+        # followed by the H2D of the step that reuses its buffer set
+        for n in range(min(nb, len(batches))):
+            h2d(n)
+        for n in range(len(batches)):
+            compute_stream.wait_event(h2d_done[n])
+            self._forward(self.sets[n % nb], compute_stream)
+            fwd_done[n].record(compute_stream)
+            d2h(n)
+            if n + nb < len(batches):
+                h2d(n + nb)
+        last = self.sets[(len(batches) - 1) % nb]
+        return last["out_host"], last["lse_host"]

@@ -119,3 +119,26 @@ def test_host_runner_end_to_end(cuda_lib):
     torch.cuda.synchronize()
     O_ref, L_ref = oracle.attention_reference(q, k, v, True, w.scale)
     assert_parity(out, lse, O_ref, L_ref, torch.bfloat16, "host runner")
+
+
+def test_host_runner_pipelined_steps(cuda_lib):
+    """Three different inputs through two buffer sets and two streams: each step's host
+    result is the oracle's for its own inputs."""
+    from sequence_exact_attention_ring_b200 import HostRunner
+    ws = [synthetic.custom("e2e", "bf16", 1, 4, 2, 1024, 128, 4, True, "striped", 31 + n) for n in range(3)]
+    inputs = [tuple(t.pin_memory() for t in synthetic.make_inputs(w, "cpu")) for w in ws]
+    r = HostRunner(inputs[0][0].shape, inputs[0][1].shape, torch.bfloat16, 4, True, "striped", ws[0].scale,
+                   buffers=2)
+    copy_stream, compute_stream = torch.cuda.Stream(), torch.cuda.Stream()
+    results = []
+    for n in range(3):  # one step at a time, keeping each result before its set is reused
+        out, lse = r.run_steps([inputs[n]], copy_stream, compute_stream)
+        copy_stream.synchronize()
+        results.append((out.clone(), lse.clone()))
+    out, lse = r.run_steps(inputs, copy_stream, compute_stream)  # all three pipelined
+    copy_stream.synchronize()
+    results.append((out.clone(), lse.clone()))
+    for n, (o, l) in enumerate(results):
+        q, k, v = inputs[min(n, 2)]
+        O_ref, L_ref = oracle.attention_reference(q, k, v, True, ws[0].scale)
+        assert_parity(o, l, O_ref, L_ref, torch.bfloat16, f"pipelined step {n}")

@@ -33,7 +33,7 @@
 // in exchange needs no atomic accumulation anywhere.
 //
 // Tensor memory (512 columns): score buffers [0,64) and [64,128), dP buffers [128,192)
-// and [192,256), accumulators from 256. Eight elementwise warps split each 64-column
+// and [192,256), accumulators from 256 (the dQ kernel keeps Q and dO at 384 and 448). Eight elementwise warps split each 64-column
 // tile: warp w owns TMEM lanes 32 (w % 4) .. +31 and columns 32 (w / 4) .. +31 of it;
 // it writes its 32 bf16 P (or dS) values packed into the first 16 of those columns,
 // which it has already read, so no warp overwrites a value another warp still needs.
@@ -125,6 +125,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint16_t* __restric
 
 struct Params {
   RingGeom g;
+  const void* q;       // bf16 [B,Hq,S,D] (read directly by the dQ kernel)
+  const void* dout;    // bf16 [B,Hq,S,D]
   const float* lse2;   // [B*Hq][P][sq_pad]
   const float* delta;  // [B*Hq][P][sq_pad]
   int64_t sq_pad;
@@ -390,14 +392,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Shared memory of the dQ kernel: Q and dO once, then a ring of 64-key K or V slots.
-constexpr int kB_OffQ = 0;
-constexpr int kB_OffDO = kTileBytes;
-constexpr int kB_OffRing = 2 * kTileBytes;
+// Shared memory of the dQ kernel: a ring of 64-key K or V slots only; Q and dO sit
+// in tensor memory as the A operands of their products.
+constexpr int kB_OffRing = 0;
 constexpr int kB_SlotsFit = (kSmemLimit - 1024 - 64 - 512 - kB_OffRing) / kStepTileBytes;
-constexpr int kB_Slots = kB_SlotsFit < 10 ? kB_SlotsFit : 10;
+constexpr int kB_Slots = kB_SlotsFit < 12 ? kB_SlotsFit : 12;
 constexpr int kB_OffBar = kB_OffRing + kB_Slots * kStepTileBytes;
-enum BarB { kB_QFull = 0, kB_SFull = 1, kB_PReady = 3, kB_Done = 5, kB_Drain = 6, kB_Ring = 7 };
+constexpr uint32_t kColQ = 384;   // Q tile, bf16 pairs: 64 columns
+constexpr uint32_t kColDO = 448;  // dO tile, bf16 pairs: 64 columns
+// kB_QReady: the eight elementwise warps have written Q and dO into tensor memory
+enum BarB { kB_QReady = 0, kB_SFull = 1, kB_PReady = 3, kB_Done = 5, kB_Drain = 6, kB_Ring = 7 };
 constexpr int kB_NumBars = kB_Ring + 2 * kB_Slots;
 constexpr int kB_OffMisc = kB_OffBar + kB_NumBars * 8;
 constexpr int kB_SmemBytes = kB_OffMisc + 64 + 1024;
@@ -405,7 +409,9 @@ static_assert(kB_Slots >= 4, "need two steps of K and V slots");
 static_assert(kB_SmemBytes <= kSmemLimit, "shared memory budget");
 
 // dQ: one CTA per 128-row query tile; keys arrive in steps of 64 along the backward
-// ring. TMEM holds two buffers of (S 64 columns, dP 64 columns) and the dQ accumulator.
+// ring. TMEM holds two buffers of (S 64 columns, dP 64 columns), the dQ accumulator,
+// and Q and dO as packed bf16 pairs: S = Q K^T and dP = dO V^T then take A from
+// tensor memory and read only the 64-key step from shared memory.
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -422,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const RingGeom& g = p.g;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars[kB_QFull], 1);
+    mbar_init(&bars[kB_QReady], kEwWarps);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars[kB_SFull + b], 1);
       mbar_init(&bars[kB_PReady + b], kEwWarps);
@@ -457,12 +463,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       int c1, c2;
-      shard_map_coords(g, U.i, a0, c1, c2);
-      mbar_arrive_expect_tx(&bars[kB_QFull], 2 * kTileBytes);
-      for (int bx = 0; bx < 2; ++bx) {
-        tma_load_4d(smem + kB_OffQ + bx * kBoxBytes, &tm_q, &bars[kB_QFull], bx * BOXW, c1, c2, bh_q);
-        tma_load_4d(smem + kB_OffDO + bx * kBoxBytes, &tm_do, &bars[kB_QFull], bx * BOXW, c1, c2, bh_q);
-      }
       int64_t m = 0;
       bool ok = true;
       for (TileWalk w = walk_begin_rev(g, U.i, a_hi, TS); walk_valid(w) && ok; walk_next(g, w, a_hi, TS)) {
@@ -478,7 +478,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (!ok) {
-        drain_wait(&bars[kB_QFull], 0, p.watchdog_ns);
         for (int64_t x = (m > kB_Slots ? m - kB_Slots : 0); x < m; ++x)
           drain_wait(&full[slot_of(x)], phase_of(x), p.watchdog_ns);
       }
@@ -487,8 +486,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------------ MMA issuer
     const bool issuer = elect_one_sync();
     const uint32_t sbase = smem_u32(smem);
-    const uint64_t dQd = smem_desc_sw128(sbase + kB_OffQ, 0, 1024);
-    const uint64_t dOd = smem_desc_sw128(sbase + kB_OffDO, 0, 1024);
     auto all = [&](bool r) { return __all_sync(0xffffffffu, r); };
     auto slot_addr = [&](int64_t m) { return sbase + kB_OffRing + slot_of(m) * kStepTileBytes; };
     // S = Q K^T and dP = dO V^T of step n into buffer n % 2
@@ -500,19 +497,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t bk = smem_desc_sw128(slot_addr(2 * n), 0, 1024);
       const uint64_t bv = smem_desc_sw128(slot_addr(2 * n + 1), 0, 1024);
 #pragma unroll
-      for (int k = 0; k < D / 16; ++k)
-        if (issuer) mma_ss(tmem + col_s(b), kmajor_step(dQd, k), kmajor64_step(bk, k), kIdescSS64, k > 0);
+      for (int k = 0; k < D / 16; ++k)  // K step k: dims 16k..16k+15 = packed columns 8k..8k+7
+        if (issuer) mma_ts(tmem + col_s(b), tmem + kColQ + 8 * k, kmajor64_step(bk, k), kIdescSS64, k > 0);
 #pragma unroll
       for (int k = 0; k < D / 16; ++k)
-        if (issuer) mma_ss(tmem + col_dp(b), kmajor_step(dOd, k), kmajor64_step(bv, k), kIdescSS64, k > 0);
+        if (issuer) mma_ts(tmem + col_dp(b), tmem + kColDO + 8 * k, kmajor64_step(bv, k), kIdescSS64, k > 0);
       if (issuer) {
         mma_commit(&bars[kB_SFull + b]);
         mma_commit(&empty[slot_of(2 * n + 1)]);  // V is no longer needed once dP is done
       }
       return true;
     };
-    bool ok = N > 0 && all(mbar_wait(&bars[kB_QFull], 0, wd));
-    if (ok) ok = issue_sd(0);
+    bool ok = N > 0 && all(mbar_wait(&bars[kB_QReady], 0, wd));
+    if (ok) {
+      tc_fence_after();
+      ok = issue_sd(0);
+    }
     if (ok && N > 1) ok = issue_sd(1);
     for (int64_t n = 0; ok && n < N; ++n) {
       const int b = (int)(n & 1);
@@ -541,6 +541,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float row_lse2 = p.lse2[stat];
     const float row_delta = p.delta[stat];
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    if (N > 0) {
+      // this thread's row, dims 64 hh .. 64 hh + 63, as 32 bf16 pairs (the memory order);
+      // rows past the shard are zeros
+      const bool row_ok = a < g.Sq;
+      const int64_t base = ((int64_t)bh_q * g.S + (row_ok ? token_of(g, U.i, a) : 0)) * D + 64 * hh;
+      uint32_t x[32];
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const uint16_t* src = static_cast<const uint16_t*>(t == 0 ? p.q : p.dout) + base;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 v4 = row_ok ? *reinterpret_cast<const uint4*>(src + 8 * c) : make_uint4(0, 0, 0, 0);
+          x[4 * c] = v4.x;
+          x[4 * c + 1] = v4.y;
+          x[4 * c + 2] = v4.z;
+          x[4 * c + 3] = v4.w;
+        }
+        tmem_st32(tmem + lane_off + (t == 0 ? kColQ : kColDO) + 32 * hh, x);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[kB_QReady]);
+    }
     int64_t n = 0;
     bool ok = true;
     for (TileWalk w = walk_begin_rev(g, U.i, a_hi, TS); walk_valid(w); walk_next(g, w, a_hi, TS), ++n) {
@@ -609,6 +633,8 @@ int launch_bwd_sm100(const void* q, const void* k, const void* v, const void* ou
   if ((rc = encode_shard_map(&mv64, v, g, g.Hkv, D, TS)) != 0) return rc;
   Params p;
   p.g = g;
+  p.q = q;
+  p.dout = dout;
   p.lse2 = lse2;
   p.delta = delta;
   p.sq_pad = sq_pad;

@@ -175,7 +175,7 @@ size_t ring_attn_decode_workspace_bytes(int B, int Hq, int Hkv, int64_t S, int D
  * the merge of ring_attn_merge.
  *   q   : device [B, Hq, D] bf16          k, v : device [B, Hkv, S, D] bf16
  *   out : device [B, Hq, D] bf16          lse  : device [B, Hq] fp32
- * Supported: bf16, D = 128, Hq/Hkv <= 16, an sm_100 device (zigzag needs
+ * Supported: bf16, D = 128, Hq/Hkv <= 32, an sm_100 device (zigzag needs
  * (S/(2P)) % 128 == 0); otherwise RING_ATTN_EUNSUPPORTED. S % P == 0.
  */
 int ring_attn_decode(const void* q, const void* k, const void* v, void* out, float* lse,

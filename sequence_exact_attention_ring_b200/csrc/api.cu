@@ -230,7 +230,7 @@ int ring_attn_decode(const void* q, const void* k, const void* v, void* out, flo
   const size_t need = ring_attn_decode_workspace_bytes(B, Hq, Hkv, S, D, P, layout, dtype);
   if (!workspace || workspace_bytes < need || !aligned16(workspace)) return RING_ATTN_EWORKSPACE;
   if (!(scale > 0.f) || !isfinite(scale)) return RING_ATTN_EINVAL;
-  if (dtype != RING_ATTN_DTYPE_BF16 || D != 128 || Hq / Hkv > 16 || !tcgen05_layout_ok(g) || !device_is_sm100())
+  if (dtype != RING_ATTN_DTYPE_BF16 || D != 128 || Hq / Hkv > 32 || !tcgen05_layout_ok(g) || !device_is_sm100())
     return RING_ATTN_EUNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if ((rc = reset_status(workspace, st))) return rc;

@@ -10,21 +10,17 @@
 // ring_attn_merge then combines the P * chunks partials with the online-softmax
 // rescale (RingAttention deep-architecture article, techknowgenie, section 3).
 //
-// Per CTA: one producer warp streams 128-key K and V tiles with TMA (the shard
-// maps, 128-byte swizzle) through a 3-stage ring; eight consumer warps then
-//   1. score: thread (half, r) forms the dot products of key r of the tile with
-//      every query head of the group over one half of the head dim (q in shared
-//      memory, read as a broadcast; the swizzle makes the lanes' reads of 32
-//      different key rows conflict-free);
-//   2. warps 0-3 add the halves, take the tile maximum per head, move the reference
-//      maximum only when it grows by more than 8 (log2 units; every consumer then
-//      rescales its O and l), and write p = 2^(s - m) to shared memory;
-//   3. accumulate: thread (half, d) adds p_key * V[key][d] over its half of the
-//      tile's keys into output column d of every head; the halves are summed once
-//      at the end of the chunk.
-// The consumer warps meet on a named barrier (they always take the same path: only
-// one thread waits on the tile's mbarrier, with the watchdog, and broadcasts the
-// outcome).
+// Per CTA, the blockwise online softmax of the forward kernels with a 128-row query
+// tile of which only the group's REP rows are real (the others are never read):
+//   warp 0  softmax and epilogue: TMEM lanes 0..31 = query heads of the group
+//   warp 1  TMA producer: 128-key K and V tiles through a 3-stage ring
+//   warp 2  TMEM owner and MMA issuer: S = Q K^T with Q in tensor memory as the A
+//           operand (so only the K tile is read from shared memory), O += P V with P
+//           in tensor memory
+// Tensor memory: S double-buffered [0,128) and [128,256), O [256,384), Q [384,448).
+// S of tile n + 1 is computed while the softmax works on tile n; the tensor work per
+// tile (about 1000 clocks) stays under the time HBM needs to deliver the tile, for
+// any group size up to 32.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -33,6 +29,7 @@
 #include "ring_schedule.h"
 #include "ringattn_internal.h"
 #include "sm100_ptx.cuh"
+#include "softmax_rows.cuh"
 
 namespace ringattn {
 namespace dec {
@@ -44,19 +41,20 @@ constexpr int kBoxBytes = TK * BOXW * 2;  // 16 KiB
 constexpr int kTileBytes = TK * D * 2;    // 32 KiB
 constexpr int kStages = 3;
 constexpr int kStageBytes = 2 * kTileBytes;  // K then V
-constexpr int kMaxRep = 16;
-constexpr int kConsumers = 256;  // 8 warps: two halves of the head dim (scores) or of the keys (P V)
-constexpr int kThreads = kConsumers + 32;
-constexpr int kProducerWarp = kConsumers / 32;
-constexpr int kOffQ = kStages * kStageBytes;              // fp32 [rep][D]
-constexpr int kOffP = kOffQ + kMaxRep * D * 4;            // fp32 [rep][TK]
-constexpr int kOffPart = kOffP + kMaxRep * TK * 4;        // fp32 [2][rep][TK] partial dots / partial O
-constexpr int kOffRed = kOffPart + 2 * kMaxRep * TK * 4;  // fp32 [2][4 warps][rep]
-constexpr int kOffBar = kOffRed + 2 * 4 * kMaxRep * 4;    // full[kStages], empty[kStages]
-constexpr int kOffMisc = kOffBar + 2 * kStages * 8;
+constexpr int kMaxRep = 32;
+constexpr int kThreads = 128;
+constexpr int kSoftmaxWarp = 0, kProducerWarp = 1, kMmaWarp = 2;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColO = 256;
+constexpr uint32_t kColQ = 384;
+constexpr uint32_t kIdescQK = idesc_bf16_f32(128, TK, 0, 0);
+constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, 0, 1);
+enum Bar { kQReady = 0, kSFull = 1, kPReady = 3, kPvDone = 5, kODone = 6, kDrain = 7, kFull = 8 };
+constexpr int kNumBars = kFull + 2 * kStages;
+constexpr int kOffBar = kStages * kStageBytes;
+constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 64 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
-constexpr float kRescaleLog2 = 8.0f;
 
 struct Params {
   RingGeom g;
@@ -70,8 +68,6 @@ struct Params {
   uint64_t watchdog_ns;
 };
 
-__device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kConsumers) : "memory"); }
-
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   const uint64_t t0 = global_timer_ns();
   while (!mbar_try_wait(bar, parity)) {
@@ -79,33 +75,18 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint6
   }
 }
 
-// Byte offset of the 8-element chunk holding column d of row r in a 128-byte-swizzled
-// tile staged as two 64-column boxes.
-__device__ __forceinline__ int swz(int r, int d) {
-  return (d / BOXW) * kBoxBytes + r * 128 + ((((d % BOXW) / 8) ^ (r & 7)) * 16);
-}
-
-__device__ __forceinline__ float bf16_lo(uint32_t x) { return __uint_as_float(x << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
-
-// REP: query heads per kv head (the GQA group size), a compile-time constant so that
-// every per-head loop is unrolled exactly.
-template <int REP>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* qs = reinterpret_cast<float*>(smem + kOffQ);
-  float* ps = reinterpret_cast<float*>(smem + kOffP);
-  float* part = reinterpret_cast<float*>(smem + kOffPart);
-  float* red = reinterpret_cast<float*>(smem + kOffRed);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kOffBar);
-  uint64_t* empty = full + kStages;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc);
-  volatile int* go = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
-  const int tid = threadIdx.x;
-  const int warp = tid / 32, lane = tid % 32;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint64_t* full = &bars[kFull];
+  uint64_t* empty = &bars[kFull + kStages];
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 8);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const RingGeom& g = p.g;
+  const int rep = g.Hq / g.Hkv;
 
   // unit: chunk fastest, then shard, then (b, kv head)
   int64_t u = blockIdx.x;
@@ -118,22 +99,36 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int bh_kv = b * g.Hkv + kvh;
   const int64_t k0 = (int64_t)c * p.chunk_keys;
   const int64_t k1 = (k0 + p.chunk_keys < g.Sq) ? k0 + p.chunk_keys : g.Sq;
-  const int ntiles = (int)((k1 - k0 + TK - 1) / TK);
+  const int ntiles = (int)((k1 - k0 + TK - 1) / TK);  // >= 1 for every launched chunk
 
-  if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kConsumers / 32);
+  if (threadIdx.x == 0) {
+    mbar_init(&bars[kQReady], 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&bars[kSFull + x], 1);
+      mbar_init(&bars[kPReady + x], 1);
     }
+    mbar_init(&bars[kPvDone], 1);
+    mbar_init(&bars[kODone], 1);
+    mbar_init(&bars[kDrain], 1);
+    for (int s = 0; s < 2 * kStages; ++s) mbar_init(&bars[kFull + s], 1);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
   const Watchdog wd{abort_flag, p.status, p.watchdog_ns};
 
   if (warp == kProducerWarp) {
     if (lane == 0) {
       // ------------------------------------------------------------------ producer
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
       bool ok = true;
       int n = 0;
       for (; n < ntiles && ok; ++n) {
@@ -153,139 +148,156 @@ __global__ void __launch_bounds__(kThreads, 1)
           drain_wait(&full[m % kStages], (uint32_t)(m / kStages) & 1, p.watchdog_ns);
       }
     }
-    return;
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------------ MMA issuer
+    const bool issuer = elect_one_sync();
+    const uint32_t sbase = smem_u32(smem);
+    auto all = [&](bool r) { return __all_sync(0xffffffffu, r); };
+    // S_b = Q K_n^T into buffer n % 2 once tile n has landed
+    auto issue_s = [&](int n) -> bool {
+      const int s = n % kStages;
+      if (!all(mbar_wait(&full[s], (uint32_t)(n / kStages) & 1, wd))) return false;
+      tc_fence_after();
+      const uint64_t dk = smem_desc_sw128(sbase + s * kStageBytes, 0, 1024);
+      const uint32_t d = tmem + (uint32_t)(128 * (n & 1));
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k)
+        if (issuer)
+          mma_ts(d, tmem + kColQ + 8 * k, dk + (uint64_t)((((k / 4) * kBoxBytes) + (k % 4) * 32) >> 4), kIdescQK,
+                 k > 0);
+      if (issuer) mma_commit(&bars[kSFull + (n & 1)]);
+      return true;
+    };
+    bool ok = all(mbar_wait(&bars[kQReady], 0, wd));
+    if (ok) {
+      tc_fence_after();
+      ok = issue_s(0);
+    }
+    if (ok && ntiles > 1) ok = issue_s(1);
+    for (int n = 0; ok && n < ntiles; ++n) {
+      const int s = n % kStages;
+      if (!(ok = all(mbar_wait(&bars[kPReady + (n & 1)], (uint32_t)((n >> 1) & 1), wd)))) break;
+      tc_fence_after();
+      // O += P V: P in the first 64 columns of S_b, V as the MN-major B operand
+      const uint64_t dv = smem_desc_sw128(sbase + s * kStageBytes + kTileBytes, kBoxBytes, 1024);
+      const uint32_t pa = tmem + (uint32_t)(128 * (n & 1));
+#pragma unroll
+      for (int k = 0; k < TK / 16; ++k)
+        if (issuer) mma_ts(tmem + kColO, pa + 8 * k, dv + (uint64_t)((k * 16 * 128) >> 4), kIdescPV, !(n == 0 && k == 0));
+      if (issuer) {
+        mma_commit(&bars[kPvDone]);
+        mma_commit(&empty[s]);
+      }
+      if (n + 2 < ntiles && !(ok = issue_s(n + 2))) break;
+    }
+    if (issuer) {
+      mma_commit(&bars[kODone]);
+      mma_commit(&bars[kDrain]);
+    }
+    drain_wait(&bars[kDrain], 0, p.watchdog_ns);
+  } else if (warp == kSoftmaxWarp) {
+    // ------------------------------------------------------------- softmax + epilogue
+    const int h = lane;                  // query head of the group (row of the tile)
+    const bool live = h < rep;
+    {
+      // Q rows into tensor memory as bf16 pairs (dims 2c, 2c + 1 in column c), zeros
+      // for the rows past the group; rows 32..127 are never read back
+      uint32_t x[32];
+      const uint16_t* src = p.q + ((int64_t)(b * g.Hq + kvh * rep + (live ? h : 0))) * D;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+          const uint4 v4 = live ? *reinterpret_cast<const uint4*>(src + 64 * half + 8 * cc) : make_uint4(0, 0, 0, 0);
+          x[4 * cc] = v4.x;
+          x[4 * cc + 1] = v4.y;
+          x[4 * cc + 2] = v4.z;
+          x[4 * cc + 3] = v4.w;
+        }
+        tmem_st32(tmem + kColQ + 32 * half, x);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[kQReady]);
+    }
+    float m_ref = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int n = 0; n < ntiles; ++n) {
+      const int bb = n & 1;
+      if (!(ok = mbar_wait(&bars[kSFull + bb], (uint32_t)((n >> 1) & 1), wd))) break;
+      tc_fence_after();
+      const uint32_t tS = tmem + (uint32_t)(128 * bb);
+      uint32_t sr[TK];
+#pragma unroll
+      for (int cc = 0; cc < TK / 32; ++cc) tmem_ld32(tS + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[cc * 32]));
+      tmem_wait_ld();
+      const int cut = live ? visible_keys<TK>(k0 + (int64_t)n * TK, k1) : 0;  // keys past the chunk are out
+      mask_scores<TK>(sr, cut);
+      const float mblk = cut == 0 ? -INFINITY : raw_rowmax<TK>(sr) * p.scale_log2;
+      float alpha = 1.f;
+      bool resc = false;
+      if (n == 0) {
+        m_ref = mblk;
+      } else if (mblk > m_ref + kRescaleLog2) {
+        alpha = (m_ref == -INFINITY) ? 0.f : ex2_approx(m_ref - mblk);
+        l *= alpha;
+        m_ref = mblk;
+        resc = true;
+      }
+      if (__any_sync(0xffffffffu, resc)) {
+        // S of this tile was issued before P V of the previous one: O must hold every
+        // product issued so far before it is rescaled
+        if (n > 0 && !(ok = mbar_wait(&bars[kPvDone], (uint32_t)((n - 1) & 1), wd))) break;
+        tc_fence_after();
+        rescale_o<D>(tmem + kColO, alpha);
+      }
+      uint32_t pk[TK / 2];
+      if (cut == 0) {
+#pragma unroll
+        for (int cc = 0; cc < TK / 2; ++cc) pk[cc] = 0u;
+      } else {
+        l += exp_pack<TK, 0>(sr, p.scale_log2, (m_ref == -INFINITY) ? 0.f : m_ref, pk);
+      }
+#pragma unroll
+      for (int cc = 0; cc < TK / 64; ++cc) tmem_st32(tS + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[cc * 32]));
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[kPReady + bb]);
+    }
+    if (ok && mbar_wait(&bars[kODone], 0, wd)) {
+      tc_fence_after();
+      const int part = j * p.chunks + c;
+      const int64_t rows = (int64_t)g.B * g.Hq;
+      const int64_t row = (int64_t)b * g.Hq + kvh * rep + (live ? h : 0);
+      const bool empty_part = !(l > 0.f);  // cannot happen for a chunk with a key; kept exact anyway
+      const float inv_l = empty_part ? 0.f : 1.f / l;
+      float* dst = p.o_parts + ((int64_t)part * rows + row) * D;
+#pragma unroll 1
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        tmem_ld32(tmem + kColO + cc * 32, o);
+        tmem_wait_ld();
+        if (live) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(dst + cc * 32 + e) =
+                make_float4(__uint_as_float(o[e]) * inv_l, __uint_as_float(o[e + 1]) * inv_l,
+                            __uint_as_float(o[e + 2]) * inv_l, __uint_as_float(o[e + 3]) * inv_l);
+        }
+      }
+      if (live)
+        p.lse_parts[(int64_t)part * rows + row] =
+            empty_part ? -INFINITY : (m_ref + log2f(l)) * 0.69314718055994530942f;
+    }
   }
 
-  // ---------------------------------------------------------------------- consumers
-  const int half = tid / TK;  // scores: half of the head dim; P V: half of the tile's keys
-  const int r = tid % TK;     // scores: key row of the tile; P V: output column
-  for (int x = tid; x < REP * D; x += kConsumers) {
-    const int h = x / D, d = x % D;
-    qs[h * D + d] = bf16_lo(p.q[((int64_t)(b * g.Hq + kvh * REP + h)) * D + d]);
-  }
-  float o[REP], m_ref[REP], l[REP], sc[REP];
-#pragma unroll
-  for (int h = 0; h < REP; ++h) {
-    o[h] = 0.f;
-    m_ref[h] = -INFINITY;
-    l[h] = 0.f;
-  }
-  bool ok = true;
-  for (int n = 0; n < ntiles; ++n) {
-    const int s = n % kStages;
-    if (tid == 0) *go = mbar_wait(&full[s], (uint32_t)(n / kStages) & 1, wd) ? 1 : 0;
-    consumers_sync();
-    if (!*go) {
-      ok = false;
-      break;
-    }
-    const uint8_t* Ks = smem + s * kStageBytes;
-    const uint8_t* Vs = Ks + kTileBytes;
-    const bool valid = k0 + (int64_t)n * TK + r < k1;
-    // 1. partial scores over this thread's half of the head dim
-    {
-      float a0[REP], a1[REP];
-#pragma unroll
-      for (int h = 0; h < REP; ++h) a0[h] = a1[h] = 0.f;
-#pragma unroll
-      for (int dd = 0; dd < D / 2; dd += 8) {
-        const int d = half * (D / 2) + dd;
-        const uint4 kk = *reinterpret_cast<const uint4*>(Ks + swz(r, d));
-#pragma unroll
-        for (int h = 0; h < REP; ++h) {
-          const float4 q0 = *reinterpret_cast<const float4*>(qs + h * D + d);
-          const float4 q1 = *reinterpret_cast<const float4*>(qs + h * D + d + 4);
-          a0[h] = fmaf(bf16_lo(kk.x), q0.x, fmaf(bf16_hi(kk.x), q0.y, fmaf(bf16_lo(kk.y), q0.z, fmaf(bf16_hi(kk.y), q0.w, a0[h]))));
-          a1[h] = fmaf(bf16_lo(kk.z), q1.x, fmaf(bf16_hi(kk.z), q1.y, fmaf(bf16_lo(kk.w), q1.z, fmaf(bf16_hi(kk.w), q1.w, a1[h]))));
-        }
-      }
-#pragma unroll
-      for (int h = 0; h < REP; ++h) part[(half * REP + h) * TK + r] = a0[h] + a1[h];
-    }
-    consumers_sync();
-    // 2. tile maximum per head (warps 0-3 hold the 128 keys)
-    if (half == 0) {
-#pragma unroll
-      for (int h = 0; h < REP; ++h) {
-        sc[h] = valid ? (part[h * TK + r] + part[(REP + h) * TK + r]) * p.scale_log2 : -INFINITY;
-        float mx = sc[h];
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        if (lane == 0) red[warp * kMaxRep + h] = mx;
-      }
-    }
-    consumers_sync();
-    // every consumer moves the reference maximum the same way; warps 0-3 write p
-#pragma unroll
-    for (int h = 0; h < REP; ++h) {
-      const float mt = fmaxf(fmaxf(red[h], red[kMaxRep + h]), fmaxf(red[2 * kMaxRep + h], red[3 * kMaxRep + h]));
-      if (n == 0) {
-        m_ref[h] = mt;
-      } else if (mt > m_ref[h] + kRescaleLog2) {
-        const float alpha = ex2_approx(m_ref[h] - mt);
-        o[h] *= alpha;
-        l[h] *= alpha;
-        m_ref[h] = mt;
-      }
-      if (half == 0) {
-        const float pe = valid ? ex2_approx(sc[h] - m_ref[h]) : 0.f;
-        ps[h * TK + r] = pe;
-        float sum = pe;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-        if (lane == 0) red[4 * kMaxRep + warp * kMaxRep + h] = sum;
-      }
-    }
-    consumers_sync();
-    // 3. O += P V: column r, keys [64 half, 64 half + 64) of the tile
-#pragma unroll
-    for (int h = 0; h < REP; ++h)
-      l[h] += (red[4 * kMaxRep + h] + red[5 * kMaxRep + h]) + (red[6 * kMaxRep + h] + red[7 * kMaxRep + h]);
-    {
-      float b0[REP], b1[REP];
-#pragma unroll
-      for (int h = 0; h < REP; ++h) b0[h] = b1[h] = 0.f;
-      const int key0 = half * (TK / 2);
-#pragma unroll 4
-      for (int kk = 0; kk < TK / 2; kk += 4) {
-        const int key = key0 + kk;
-        float vv[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          vv[e] = bf16_lo(*reinterpret_cast<const uint16_t*>(Vs + swz(key + e, r) + (r % 8) * 2));
-#pragma unroll
-        for (int h = 0; h < REP; ++h) {
-          const float4 pp = *reinterpret_cast<const float4*>(ps + h * TK + key);
-          b0[h] = fmaf(pp.x, vv[0], fmaf(pp.y, vv[1], b0[h]));
-          b1[h] = fmaf(pp.z, vv[2], fmaf(pp.w, vv[3], b1[h]));
-        }
-      }
-#pragma unroll
-      for (int h = 0; h < REP; ++h) o[h] += b0[h] + b1[h];
-    }
-    consumers_sync();  // every consumer is done with this stage and with ps, part, red
-    if (lane == 0) mbar_arrive(&empty[s]);
-  }
-  if (!ok) return;
-  // the two key halves' partial O, then the normalised partial of this chunk
-  if (half == 1) {
-#pragma unroll
-    for (int h = 0; h < REP; ++h) part[h * TK + r] = o[h];
-  }
-  consumers_sync();
-  if (half == 0) {
-    const int pidx = j * p.chunks + c;
-    const int64_t rows = (int64_t)g.B * g.Hq;
-#pragma unroll
-    for (int h = 0; h < REP; ++h) {
-      const int64_t row = (int64_t)b * g.Hq + kvh * REP + h;
-      const float ot = o[h] + part[h * TK + r];
-      const bool empty_part = !(l[h] > 0.f);  // cannot happen for a chunk with a key; kept exact anyway
-      p.o_parts[((int64_t)pidx * rows + row) * D + r] = empty_part ? 0.f : ot / l[h];
-      if (r == 0)
-        p.lse_parts[(int64_t)pidx * rows + row] =
-            empty_part ? -INFINITY : (m_ref[h] + log2f(l[h])) * 0.69314718055994530942f;
-    }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
   }
 }
 
@@ -317,7 +329,7 @@ int launch_decode_sm100(const void* q, const void* k, const void* v, void* out, 
                         float scale, float* o_parts, float* lse_parts, int* status, uint64_t watchdog_ns,
                         cudaStream_t stream) {
   using namespace dec;
-  if (g.D != D) return RING_ATTN_EUNSUPPORTED;
+  if (g.D != D || g.Hq / g.Hkv > kMaxRep) return RING_ATTN_EUNSUPPORTED;
   int chunks = 1;
   const int chunk_tiles = decode_chunking(g, &chunks);
   if ((int64_t)g.P * chunks > 1024) return RING_ATTN_EUNSUPPORTED;
@@ -337,22 +349,9 @@ int launch_decode_sm100(const void* q, const void* k, const void* v, void* out, 
   p.watchdog_ns = watchdog_ns;
   const int64_t grid = (int64_t)g.B * g.Hkv * g.P * chunks;
   if (grid > 0x7fffffff) return RING_ATTN_EINVAL;
-  void (*kern)(CUtensorMap, CUtensorMap, Params) = nullptr;
-  switch (g.Hq / g.Hkv) {
-    case 1: kern = decode_kernel<1>; break;
-    case 2: kern = decode_kernel<2>; break;
-    case 3: kern = decode_kernel<3>; break;
-    case 4: kern = decode_kernel<4>; break;
-    case 5: kern = decode_kernel<5>; break;
-    case 6: kern = decode_kernel<6>; break;
-    case 7: kern = decode_kernel<7>; break;
-    case 8: kern = decode_kernel<8>; break;
-    case 16: kern = decode_kernel<16>; break;
-    default: return RING_ATTN_EUNSUPPORTED;
-  }
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess)
+  if (cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess)
     return RING_ATTN_ECUDA;
-  kern<<<(unsigned)grid, kThreads, kSmemBytes, stream>>>(mk, mv, p);
+  decode_kernel<<<(unsigned)grid, kThreads, kSmemBytes, stream>>>(mk, mv, p);
   if (cudaGetLastError() != cudaSuccess) return RING_ATTN_ECUDA;
   return launch_merge(o_parts, lse_parts, g.P * chunks, (int64_t)g.B * g.Hq, D, out, lse, RING_ATTN_DTYPE_BF16,
                       stream);

@@ -17,6 +17,8 @@ CASES = [
     (1, 2, 2, 1024, 4, "striped"),
     (2, 8, 2, 3000, 3, "contiguous"),   # Sq = 1000: ragged last tile of every shard
     (1, 16, 1, 2048, 8, "zigzag"),      # C = 128; 16 query heads share one kv head
+    (2, 64, 2, 1536, 3, "striped"),     # 32 query heads per kv head (the largest group)
+    (1, 4, 1, 640, 5, "contiguous"),    # Sq = 128: one tile per shard
     (1, 4, 4, 512, 1, "contiguous"),    # P = 1
     (1, 8, 8, 65536, 32, "striped"),
 ]

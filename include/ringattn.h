@@ -146,12 +146,12 @@ size_t ring_attn_bwd_workspace_bytes(int B, int Hq, int Hkv, int64_t S, int D, i
  *   P = exp(scale q k^T - lse) on the mask,  dv = P^T dout,  dP = dout v^T,
  *   Delta = rowsum(dout * out),  dS = P * (dP - Delta),
  *   dq = scale dS k,  dk = scale dS^T q   (GQA: dk, dv sum over the group's heads).
- *   q, out, dout, dq : device [B,Hq,S,D] bf16       k, v, dk, dv : device [B,Hkv,S,D] bf16
+ *   q, out, dout, dq : device [B,Hq,S,D] in dtype    k, v, dk, dv : device [B,Hkv,S,D] in dtype
  *   lse              : device [B,Hq,S] fp32 as returned by ring_attn_fwd
  *   workspace        : >= ring_attn_bwd_workspace_bytes(); first word is the status word
- * Supported: dtype bf16, D = 128, an sm_100 device (zigzag needs (S/(2P)) % 128 == 0);
- * otherwise RING_ATTN_EUNSUPPORTED. Outputs must not alias inputs. Same argument
- * and watchdog rules as ring_attn_fwd.
+ * bf16 with D = 128 runs on the tcgen05 kernels (zigzag: when (S/(2P)) % 128 == 0);
+ * every other dtype/D/layout the forward accepts runs on fp32 CUDA-core kernels.
+ * Outputs must not alias inputs. Same argument and watchdog rules as ring_attn_fwd.
  */
 int ring_attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
                   const void* dout, void* dq, void* dk, void* dv,

@@ -203,13 +203,15 @@ int ring_attn_bwd(const void* q, const void* k, const void* v, const void* out, 
   const size_t need = ring_attn_bwd_workspace_bytes(B, Hq, Hkv, S, D, P, causal, layout, dtype);
   if (!workspace || workspace_bytes < need || !aligned16(workspace)) return RING_ATTN_EWORKSPACE;
   if (!(scale > 0.f) || !isfinite(scale)) return RING_ATTN_EINVAL;
-  if (dtype != RING_ATTN_DTYPE_BF16 || D != 128 || !tcgen05_layout_ok(g) || !device_is_sm100())
-    return RING_ATTN_EUNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if ((rc = reset_status(workspace, st))) return rc;
   float* stats = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kWorkspaceHeaderBytes);
-  return launch_bwd_sm100(q, k, v, out, lse, dout, dq, dk, dv, g, scale, stats, static_cast<int*>(workspace),
-                          watchdog_ns(), st);
+  // bf16 with D = 128 runs on the tensor-core kernels; every other shape (fp32, D = 64,
+  // zigzag chunks that are not whole 128-row tiles) on the CUDA-core kernels
+  if (dtype == RING_ATTN_DTYPE_BF16 && D == 128 && tcgen05_layout_ok(g) && device_is_sm100())
+    return launch_bwd_sm100(q, k, v, out, lse, dout, dq, dk, dv, g, scale, stats, static_cast<int*>(workspace),
+                            watchdog_ns(), st);
+  return launch_bwd_simt(q, k, v, out, lse, dout, dq, dk, dv, g, scale, dtype, stats, st);
 }
 
 size_t ring_attn_decode_workspace_bytes(int B, int Hq, int Hkv, int64_t S, int D, int P, int layout, int dtype) {

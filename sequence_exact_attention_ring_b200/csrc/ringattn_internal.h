@@ -53,6 +53,12 @@ int launch_decode_sm100(const void* q, const void* k, const void* v, void* out, 
                         float scale, float* o_parts, float* lse_parts, int* status, uint64_t watchdog_ns,
                         cudaStream_t stream);
 
+// CUDA-core backward for the shapes the tensor-core kernels do not take (fp32 or
+// bf16, D = 64 or 128, any layout); same statistics layout in `stats`.
+int launch_bwd_simt(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dout,
+                    void* dq, void* dk, void* dv, const RingGeom& g, float scale, int dtype, float* stats,
+                    cudaStream_t stream);
+
 int launch_merge(const float* o_parts, const float* lse_parts, int n_parts, int64_t rows, int D, void* out,
                  float* lse_out, int out_dtype, cudaStream_t stream);
 

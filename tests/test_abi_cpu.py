@@ -233,5 +233,5 @@ def test_backward_workspace_and_argument_errors(lib):
     bad[17] = -0.5  # scale
     assert B.ring_attn_bwd(*bad) == B.EINVAL
     bad = list(args)
-    bad[18] = 0  # fp32: no backward kernel
+    bad[13] = 96  # head dim outside {64, 128}
     assert B.ring_attn_bwd(*bad) == B.EUNSUPPORTED

@@ -95,8 +95,30 @@ def test_backward_16k_sampled(cuda_lib, name):
     assert np.abs(sk).max() <= 2e-2 * dk.double().abs().sum(dim=2).max().item()
 
 
-def test_backward_refuses_untileable_zigzag(cuda_lib):
-    w, q, k, v, dout, out, lse = make(1, 2, 2, 1000, 128, 4, True, "zigzag", seed=221)
-    with pytest.raises(binding.RingAttnError) as e:
-        ring_attention_backward(q, k, v, out, lse, dout, w.P, True, "zigzag", w.scale)
-    assert e.value.code == binding.EUNSUPPORTED
+# shapes the tensor-core kernels do not take run on the CUDA-core backward
+SIMT_CASES = [
+    # (B, Hq, Hkv, S, D, P, causal, layout, dtype)
+    (1, 2, 2, 1000, 128, 4, True, "zigzag", "bf16"),     # C = 125: not whole 128-row tiles
+    (1, 4, 2, 768, 64, 3, True, "striped", "bf16"),      # D = 64
+    (1, 2, 1, 640, 64, 4, True, "contiguous", "fp32"),   # fp32, ragged Sq = 160
+    (2, 2, 2, 512, 128, 2, False, "striped", "fp32"),
+]
+
+
+@pytest.mark.parametrize("case", SIMT_CASES, ids=lambda c: "-".join(map(str, c)))
+def test_backward_cuda_core_path(cuda_lib, case):
+    B, Hq, Hkv, S, D, P, causal, layout, dtype = case
+    w = synthetic.custom("bwd", dtype, B, Hq, Hkv, S, D, P, causal, layout, 231)
+    q, k, v = (t.cuda() for t in synthetic.make_inputs(w, "cpu"))
+    dout = synthetic.make_dout(w, "cpu").cuda()
+    out, lse = ring_attention(q, k, v, P, causal, layout, w.scale)
+    dq, dk, dv = ring_attention_backward(q, k, v, out, lse, dout, P, causal, layout, w.scale)
+    torch.cuda.synchronize()
+    ref = oracle.attention_backward_reference(q.cpu(), k.cpu(), v.cpu(), dout.cpu(), causal, w.scale)
+    for name, got, r in zip(("dq", "dk", "dv"), (dq, dk, dv), ref):
+        if dtype == "fp32":
+            # fp32 throughout (exact exp2f, no rounded P): relative to the largest gradient
+            g = got.cpu().numpy().astype(np.float64)
+            assert np.abs(g - r).max() <= 1e-4 * np.abs(r).max(), f"{case} {name}"
+        else:
+            assert_grad(got, r, f"{case} {name}")

@@ -105,6 +105,10 @@ WORKLOADS = {
     "z5_bf16_s1m_zigzag": Workload("z5_bf16_s1m_zigzag", "bf16", 1, 8, 8, 1048576, 128, 32, True,
                                    "zigzag", 7, gen_device="cuda",
                                    description="bf16 S=1048576 P=32 causal zigzag"),
+    # head dim 64 (the single-CTA tensor-core kernel), same token count and FLOPs as the 128k case
+    "d64_bf16_s128k_striped": Workload("d64_bf16_s128k_striped", "bf16", 1, 16, 16, 131072, 64, 32, True,
+                                       "striped", 8, gen_device="cuda",
+                                       description="bf16 S=131072 Hq=16 D=64 P=32 causal striped"),
     # profiling stand-in: the 1M workload's shape at 1/8 the length (inputs 0.4 GB > L2,
     # ~45 ms per launch) so an ncu capture of every section ends in a minute or two
     "prof_bf16_s128k_striped": Workload("prof_bf16_s128k_striped", "bf16", 1, 8, 8, 131072, 128, 32, True,

@@ -328,13 +328,6 @@ __device__ __forceinline__ void mma_commit_2sm(uint64_t* bar, uint16_t cta_mask)
       : "memory");
 }
 
-// Makes this thread's ordinary shared-memory stores visible to the tensor cores and
-// TMA (the async proxy); issue it after the stores and before the signal that hands
-// the data to an MMA.
-__device__ __forceinline__ void fence_proxy_async_shared() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 // True in exactly one active lane of a converged warp (elect.sync). Code that issues
 // tcgen05 instructions runs warp-wide and guards only the issuing instruction with
 // this predicate, so descriptor arithmetic stays in warp-uniform registers.

@@ -24,7 +24,7 @@ Sources (the RingAttention pages):
          names zigzag without defining it; the plainest reading taken here cuts the
          sequence into 2P equal chunks and gives shard i chunks i and 2P-1-i.
 
-Readings where the pages are silent (each also listed in the design doc):
+Readings where the pages are silent:
   * lse = m + ln(l): natural log, in units of the scaled scores.
   * The causal diagonal is inclusive: key u is allowed for query t iff u <= t.
   * GQA: query head h reads kv head h // (Hq // Hkv).

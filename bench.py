@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synthetic.WORKLOADS))
+    ap.add_argument("--algo", default="auto", choices=["auto", "tcgen05", "tcgen05_1sm", "simt"],
+                    help="forward kernel (auto: the library's choice for the workload)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
@@ -277,7 +279,8 @@ def run_ours(args, world, rank, local):
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        ring_attention(q, k, v, w.P, w.causal, w.layout, w.scale, out=out, lse=lse, workspace=ws, stream=stream)
+        ring_attention(q, k, v, w.P, w.causal, w.layout, w.scale, out=out, lse=lse, workspace=ws, stream=stream,
+                       algo=args.algo)
 
     for _ in range(args.warmup):
         flush_l2(l2buf)

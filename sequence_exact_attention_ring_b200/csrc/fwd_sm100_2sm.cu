@@ -50,8 +50,12 @@ constexpr int kProducerWarp = 8;
 #endif
 constexpr uint32_t kProducerSleepNs = RING_ATTN_PRODUCER_SLEEP_NS;  // the producer polls slots this often
 constexpr int kMmaWarp = 9;
+// Of every 8 column pairs of a score row, this many take 2^x from the FMA-pipe
+// polynomial (exp2_poly2) and the rest from the MUFU ex2 unit. On the 1M-token
+// causal workload 2 of 8 measured 1030 TFLOP/s against 1003 with MUFU alone (the
+// exponentials are evaluated in phases, exp_pack_phased); 3 of 8 measured 1011.
 #ifndef RING_ATTN_EMU_PAIRS_PER8
-#define RING_ATTN_EMU_PAIRS_PER8 0
+#define RING_ATTN_EMU_PAIRS_PER8 2
 #endif
 constexpr int kEmuPairsPer8 = RING_ATTN_EMU_PAIRS_PER8;
 #ifndef RING_ATTN_MMA_SPIN
@@ -332,7 +336,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < BN / 2; ++c) pk[c] = 0u;
       } else {
-        l += exp_pack<BN, kEmuPairsPer8>(sr, p.scale_log2, (m_ref == NEG_INF) ? 0.f : m_ref, pk);
+        l += exp_pack_phased<BN, kEmuPairsPer8>(sr, p.scale_log2, (m_ref == NEG_INF) ? 0.f : m_ref, pk);
       }
 #pragma unroll
       for (int c = 0; c < BN / 64; ++c) tmem_st32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[c * 32]));

@@ -85,6 +85,49 @@ __device__ __forceinline__ float exp_pack(const uint32_t (&sr)[N], float scale_l
   return t0 + t1;
 }
 
+// The same result as exp_pack, written in three phases over all N scores: every
+// exponent argument first (packed FMA), then every 2^x back to back, then the bf16
+// packing and the row sum. The exponentials of a thread are independent, so the
+// phases give the scheduler long runs of independent special-function operations
+// instead of short dependent chains per column pair. Of every 8 column pairs, kEmu
+// take 2^x from the FMA-pipe polynomial (interleaved with the MUFU operations).
+template <int N, int kEmu>
+__device__ __forceinline__ float exp_pack_phased(uint32_t (&sr)[N], float scale_log2, float m_sub,
+                                                 uint32_t (&pk)[N / 2]) {
+  const uint64_t c2 = f2_splat(scale_log2);
+  const uint64_t negm = f2_splat(-m_sub);
+#pragma unroll
+  for (int c = 0; c < N; c += 2) {
+    const uint64_t xy = f2_fma(f2_pack(sr[c], sr[c + 1]), c2, negm);
+    float x0, x1;
+    f2_unpack(xy, x0, x1);
+    sr[c] = __float_as_uint(x0);
+    sr[c + 1] = __float_as_uint(x1);
+  }
+#pragma unroll
+  for (int c = 0; c < N; c += 2) {
+    if ((c / 2) % 8 < kEmu) {
+      float p0, p1;
+      f2_unpack(exp2_poly2(f2_pack(sr[c], sr[c + 1])), p0, p1);
+      sr[c] = __float_as_uint(p0);
+      sr[c + 1] = __float_as_uint(p1);
+    } else {
+      sr[c] = __float_as_uint(ex2_approx(__uint_as_float(sr[c])));
+      sr[c + 1] = __float_as_uint(ex2_approx(__uint_as_float(sr[c + 1])));
+    }
+  }
+  uint64_t acc[4] = {0, 0, 0, 0};
+#pragma unroll
+  for (int c = 0; c < N; c += 2) {
+    acc[(c / 2) % 4] = f2_add(acc[(c / 2) % 4], f2_pack(sr[c], sr[c + 1]));
+    pk[c / 2] = pack_bf16x2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+  }
+  const uint64_t t = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+  float t0, t1;
+  f2_unpack(t, t0, t1);
+  return t0 + t1;
+}
+
 // Multiplies kCols accumulator columns of this warp's 32 rows in tensor memory by
 // each lane's alpha (1 for rows that keep their reference maximum).
 template <int kCols>

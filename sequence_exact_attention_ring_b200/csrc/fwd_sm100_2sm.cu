@@ -51,13 +51,18 @@ constexpr int kProducerWarp = 8;
 constexpr uint32_t kProducerSleepNs = RING_ATTN_PRODUCER_SLEEP_NS;  // the producer polls slots this often
 constexpr int kMmaWarp = 9;
 // Of every 8 column pairs of a score row, this many take 2^x from the FMA-pipe
-// polynomial (exp2_poly2) and the rest from the MUFU ex2 unit. On the 1M-token
-// causal workload 2 of 8 measured 1030 TFLOP/s against 1003 with MUFU alone (the
-// exponentials are evaluated in phases, exp_pack_phased); 3 of 8 measured 1011.
+// polynomial (exp2_poly2) and the rest from the MUFU ex2 unit (the exponentials are
+// evaluated in phases, exp_pack_phased). On the 1M-token causal workload, with the
+// speculative exponentials below: 1 of 8 measured 1015 TFLOP/s, 2 of 8 1003, 3 of 8 988,
+// 4 of 8 938 (one box, 1462 MHz).
 #ifndef RING_ATTN_EMU_PAIRS_PER8
-#define RING_ATTN_EMU_PAIRS_PER8 2
+#define RING_ATTN_EMU_PAIRS_PER8 1
 #endif
 constexpr int kEmuPairsPer8 = RING_ATTN_EMU_PAIRS_PER8;
+#ifndef RING_ATTN_SPEC_EXP
+#define RING_ATTN_SPEC_EXP 1
+#endif
+constexpr float kSpecMaxSum = 1048576.0f;  // 2^20
 #ifndef RING_ATTN_MMA_SPIN
 #define RING_ATTN_MMA_SPIN 0
 #endif
@@ -318,25 +323,47 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mask_scores<BN>(sr, cut);
       // a block no row of this warp can see contributes nothing: P = 0, state unchanged
       const bool warp_empty = __all_sync(0xffffffffu, cut == 0);
-      const float mblk = warp_empty ? -INFINITY : raw_rowmax<BN>(sr) * p.scale_log2;
-      float alpha = 1.f;
-      bool resc = false;
-      if (n == 0) {
-        m_ref = mblk;
-      } else if (mblk > m_ref + kRescaleLog2) {
-        alpha = (m_ref == NEG_INF) ? 0.f : ex2_approx(m_ref - mblk);
-        l *= alpha;
-        m_ref = mblk;
-        resc = true;
-      }
-      // S ready for tile n implies PV(n-1) of this query tile completed: O is stable
-      if (__any_sync(0xffffffffu, resc)) rescale_o<D>(tO, alpha);
       uint32_t pk[BN / 2];
       if (warp_empty) {
 #pragma unroll
         for (int c = 0; c < BN / 2; ++c) pk[c] = 0u;
       } else {
-        l += exp_pack_phased<BN, kEmuPairsPer8>(sr, p.scale_log2, (m_ref == NEG_INF) ? 0.f : m_ref, pk);
+        float lb = 0.f;
+#if RING_ATTN_SPEC_EXP
+        // Exponentials against the current reference maximum first. The reference moves
+        // only when a block's scores rise well above it, and O/l and lse do not depend on
+        // it, so a block whose row sums stay <= kSpecMaxSum (every P <= 2^20, finite) is
+        // kept as is. Otherwise (and for the first block) the warp reloads the scores,
+        // takes the block maximum and follows the rescale rule below.
+        bool fast = __all_sync(0xffffffffu, m_ref != NEG_INF);
+        if (fast) {
+          lb = exp_pack_phased<BN, kEmuPairsPer8>(sr, p.scale_log2, m_ref, pk);
+          fast = __all_sync(0xffffffffu, lb <= kSpecMaxSum);
+        }
+        if (!fast) {
+#pragma unroll
+          for (int c = 0; c < BN / 32; ++c)
+            tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+          tmem_wait_ld();
+          mask_scores<BN>(sr, cut);
+#else
+        {
+#endif
+          const float mblk = raw_rowmax<BN>(sr) * p.scale_log2;
+          float alpha = 1.f;
+          bool resc = false;
+          if (mblk > m_ref + kRescaleLog2) {
+            // (m_ref = -inf: nothing has been accumulated yet, alpha = 0 keeps l and O at 0)
+            alpha = (m_ref == NEG_INF) ? 0.f : ex2_approx(m_ref - mblk);
+            l *= alpha;
+            m_ref = mblk;
+            resc = true;
+          }
+          // S ready for tile n implies PV(n-1) of this query tile completed: O is stable
+          if (__any_sync(0xffffffffu, resc)) rescale_o<D>(tO, alpha);
+          lb = exp_pack_phased<BN, kEmuPairsPer8>(sr, p.scale_log2, (m_ref == NEG_INF) ? 0.f : m_ref, pk);
+        }
+        l += lb;
       }
 #pragma unroll
       for (int c = 0; c < BN / 64; ++c) tmem_st32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[c * 32]));

@@ -498,13 +498,15 @@ __device__ __forceinline__ void regs_decrease() {
 // Range reduction x = n + f with n = round(x) (the 1.5*2^23 rounding trick, which
 // leaves n in the low mantissa bits of t), f in [-1/2, 1/2]; 2^f by the degree-3
 // polynomial of exp2_poly.h (constant term exactly 1); 2^n by adding n to the
-// exponent field. Inputs are clamped to >= -127, where the result is exactly +0
-// (so -inf maps to 0). Valid for x <= 127; relative error <= kExp2MaxRelErr.
+// exponent field. Inputs are clamped to [-127, 127]: below, the result is exactly +0
+// (so -inf maps to 0); above, it is 2^127 (finite, so a caller that sums the results
+// sees a huge value instead of a wrapped exponent field). Relative error <=
+// kExp2MaxRelErr on [-126, 127].
 __device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
   float a, b;
   f2_unpack(x2, a, b);
-  a = fmaxf(a, -127.f);
-  b = fmaxf(b, -127.f);
+  a = fminf(fmaxf(a, -127.f), 127.f);
+  b = fminf(fmaxf(b, -127.f), 127.f);
   const uint64_t xc = f2_pack(__float_as_uint(a), __float_as_uint(b));
   const uint64_t magic = f2_splat(12582912.0f);  // 1.5 * 2^23
   const uint64_t t = f2_add(xc, magic);

@@ -37,3 +37,13 @@ def test_special_values(cuda_lib):
     assert y[0].item() == 0.0 and y[1].item() == 0.0 and y[2].item() == 0.0
     assert y[3].item() == 1.0 and y[4].item() == 2.0 and y[5].item() == 256.0
     assert abs(y[6].item() / 2 ** -0.5 - 1) <= BOUND and abs(y[7].item() / 2 ** 0.5 - 1) <= BOUND
+
+
+def test_large_arguments_saturate_at_2_pow_127(cuda_lib):
+    """Above 127 the exponent field would wrap; the polynomial clamps, so a row sum of its
+    results shows the overflow instead of hiding it."""
+    x = torch.tensor([127.0, 128.0, 200.0, 1000.0, math.inf, 126.0], dtype=torch.float32)
+    y = run(x)
+    for v in y[:5].tolist():
+        assert v == 2.0 ** 127
+    assert y[5].item() == 2.0 ** 126

@@ -79,6 +79,7 @@ constexpr int kMmaWarp = 9;
 #define RING_ATTN_EMU_PAIRS_PER8 0
 #endif
 constexpr int kEmuPairsPer8 = RING_ATTN_EMU_PAIRS_PER8;
+constexpr float kSpecMaxSum = 1048576.0f;  // 2^20: the speculative exponentials' row-sum limit
 
 template <int D>
 struct Cfg {
@@ -333,25 +334,42 @@ __global__ void __launch_bounds__(kThreads, 1)
       mask_scores<BN>(sr, cut);
       // a block no row of this warp can see contributes nothing: P = 0, state unchanged
       const bool warp_empty = __all_sync(0xffffffffu, cut == 0);
-      const float mblk = warp_empty ? -INFINITY : raw_rowmax<BN>(sr) * p.scale_log2;
-      float alpha = 1.f;
-      bool resc = false;
-      if (n == 0) {
-        m_ref = mblk;
-      } else if (mblk > m_ref + kRescaleLog2) {
-        alpha = (m_ref == NEG_INF) ? 0.f : ex2_approx(m_ref - mblk);
-        l *= alpha;
-        m_ref = mblk;
-        resc = true;
-      }
-      // S ready for tile n implies PV(n-1) of this query tile completed: O is stable
-      if (__any_sync(0xffffffffu, resc)) rescale_o<D>(tO, alpha);
       uint32_t pk[BN / 2];
       if (warp_empty) {
 #pragma unroll
         for (int c = 0; c < BN / 2; ++c) pk[c] = 0u;
       } else {
-        l += exp_pack<BN, kEmuPairsPer8>(sr, p.scale_log2, (m_ref == NEG_INF) ? 0.f : m_ref, pk);
+        // Exponentials against the current reference maximum first (O/l and lse do not
+        // depend on it); a block whose row sums stay <= kSpecMaxSum (every P <= 2^20,
+        // finite) is kept. Otherwise, and for the first block, the warp reloads the
+        // scores, takes the block maximum and follows the rescale rule.
+        float lb = 0.f;
+        bool fast = __all_sync(0xffffffffu, m_ref != NEG_INF);
+        if (fast) {
+          lb = exp_pack_phased<BN, kEmuPairsPer8>(sr, p.scale_log2, m_ref, pk);
+          fast = __all_sync(0xffffffffu, lb <= kSpecMaxSum);
+        }
+        if (!fast) {
+#pragma unroll
+          for (int c = 0; c < BN / 32; ++c)
+            tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+          tmem_wait_ld();
+          mask_scores<BN>(sr, cut);
+          const float mblk = raw_rowmax<BN>(sr) * p.scale_log2;
+          float alpha = 1.f;
+          bool resc = false;
+          if (mblk > m_ref + kRescaleLog2) {
+            // (m_ref = -inf: nothing has been accumulated yet, alpha = 0 keeps l and O at 0)
+            alpha = (m_ref == NEG_INF) ? 0.f : ex2_approx(m_ref - mblk);
+            l *= alpha;
+            m_ref = mblk;
+            resc = true;
+          }
+          // S ready for tile n implies PV(n-1) of this query tile completed: O is stable
+          if (__any_sync(0xffffffffu, resc)) rescale_o<D>(tO, alpha);
+          lb = exp_pack_phased<BN, kEmuPairsPer8>(sr, p.scale_log2, (m_ref == NEG_INF) ? 0.f : m_ref, pk);
+        }
+        l += lb;
       }
 #pragma unroll
       for (int c = 0; c < BN / 64; ++c) tmem_st32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[c * 32]));

@@ -114,3 +114,26 @@ def test_large_configs_sampled_rows(cuda_lib, name):
     qh, kh, vh = q.cpu(), k.cpu(), v.cpu()
     O_ref, L_ref = oracle.attention_rows(qh, kh, vh, rows, w.causal, w.scale)
     assert_parity(o_s, l_s, O_ref, L_ref, torch.bfloat16, name)
+
+
+@pytest.mark.parametrize("D,algo", [(128, "tcgen05"), (64, "tcgen05"), (128, "tcgen05_1sm")])
+@pytest.mark.parametrize("pattern", ["rising", "jump"])
+def test_reference_maximum_moves(cuda_lib, D, algo, pattern):
+    """Scores that climb along the sequence (the running maximum moves again and again), or
+    a few keys whose scores jump far past 2^127 relative to the running maximum (one block's
+    exponentials overflow): the kernels exponentiate against the running maximum first and
+    must fall back to the block maximum and rescale O and l."""
+    w = synthetic.custom("mx", "bf16", 1, 2, 2, 2048, D, 4, True, "striped", 41)
+    q, k, v = synthetic.make_inputs(w, "cpu")
+    kf = k.float()
+    if pattern == "rising":
+        kf = kf * (1.0 + 6.0 * torch.arange(w.S, dtype=torch.float32) / w.S)[None, None, :, None]
+    else:
+        idx = torch.randperm(w.S, generator=torch.Generator().manual_seed(5))[:8]
+        kf[:, :, idx] *= 128.0
+    k = kf.to(torch.bfloat16)
+    q, k, v = q.cuda(), k.cuda(), v.cuda()
+    out, lse = ring_attention(q, k, v, w.P, True, "striped", w.scale, algo=algo)
+    torch.cuda.synchronize()
+    O_ref, L_ref = oracle.attention_reference(q.cpu(), k.cpu(), v.cpu(), True, w.scale)
+    assert_parity(out, lse, O_ref, L_ref, torch.bfloat16, f"{pattern} D={D} {algo}")

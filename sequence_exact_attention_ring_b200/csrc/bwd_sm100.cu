@@ -138,28 +138,41 @@ struct Params {
   uint64_t watchdog_ns;
 };
 
-// P and dS for 32 columns: s, dp raw fp32 bits; stat_lse2/stat_delta per column (or
-// broadcast); columns c < cmin (or c >= cmax) are masked to P = 0.
-__device__ __forceinline__ void p_ds_chunk(const uint32_t (&s)[32], const uint32_t (&dp)[32], const float* lse2c,
-                                           const float* deltac, float row_lse2, float row_delta, bool per_col,
-                                           float scale_log2, int c0, int cmin, int cmax, uint32_t* pp,
-                                           uint32_t* pds) {
+// P and dS for 32 columns (raw fp32 bits of s and dP), on packed column pairs (f32x2
+// arithmetic): x = s * scale_log2 - lse2,
+// P = 2^x, dS = P * (dP - Delta). kPerCol: the statistics belong to the columns (read in
+// pairs from shared memory); otherwise one row value for all columns. The per-column mask
+// selects run only when a column of the chunk lies outside [cmin, cmax).
+template <bool kPerCol>
+__device__ __forceinline__ void p_ds_chunk_packed(const uint32_t (&s)[32], const uint32_t (&dp)[32],
+                                                  const float* lse2c, const float* deltac, float row_lse2,
+                                                  float row_delta, float scale_log2, int c0, int cmin, int cmax,
+                                                  uint32_t* pp, uint32_t* pds) {
+  const uint64_t c2 = f2_splat(scale_log2);
+  const uint64_t l2r = f2_splat(row_lse2);
+  const uint64_t dlr = f2_splat(row_delta);
+  const bool whole = c0 >= cmin && c0 + 32 <= cmax;
 #pragma unroll
   for (int e = 0; e < 32; e += 2) {
-    float pv[2], dv[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int c = c0 + e + h;
-      const float l2 = per_col ? lse2c[e + h] : row_lse2;
-      const float dl = per_col ? deltac[e + h] : row_delta;
-      const bool on = c >= cmin && c < cmax;
-      const float x = fmaf(__uint_as_float(s[e + h]), scale_log2, -l2);
-      const float pe = on ? ex2_approx(x) : 0.f;
-      pv[h] = pe;
-      dv[h] = pe * (__uint_as_float(dp[e + h]) - dl);
+    uint64_t l2 = l2r, dl = dlr;
+    if (kPerCol) {
+      const float2 lv = *reinterpret_cast<const float2*>(lse2c + e);
+      const float2 dv = *reinterpret_cast<const float2*>(deltac + e);
+      l2 = f2_pack(__float_as_uint(lv.x), __float_as_uint(lv.y));
+      dl = f2_pack(__float_as_uint(dv.x), __float_as_uint(dv.y));
     }
-    pp[e / 2] = pack_bf16x2(pv[0], pv[1]);
-    pds[e / 2] = pack_bf16x2(dv[0], dv[1]);
+    float x0, x1;
+    f2_unpack(f2_sub(f2_mul(f2_pack(s[e], s[e + 1]), c2), l2), x0, x1);
+    float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+    if (!whole) {
+      p0 = (c0 + e >= cmin && c0 + e < cmax) ? p0 : 0.f;
+      p1 = (c0 + e + 1 >= cmin && c0 + e + 1 < cmax) ? p1 : 0.f;
+    }
+    const uint64_t pv = f2_pack(__float_as_uint(p0), __float_as_uint(p1));
+    float d0, d1;
+    f2_unpack(f2_mul(pv, f2_sub(f2_pack(dp[e], dp[e + 1]), dl)), d0, d1);
+    pp[e / 2] = pack_bf16x2(p0, p1);
+    pds[e / 2] = pack_bf16x2(d0, d1);
   }
 }
 
@@ -363,8 +376,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld32(tmem + lane_off + col_s(b) + 32 * hh, sv);
       tmem_ld32(tmem + lane_off + col_dp(b) + 32 * hh, dpv);
       tmem_wait_ld();
-      p_ds_chunk(sv, dpv, lse2c + 32 * hh, deltac + 32 * hh, 0.f, 0.f, true, p.scale_log2, 32 * hh, cmin, TS, pp,
-                 pds);
+      p_ds_chunk_packed<true>(sv, dpv, lse2c + 32 * hh, deltac + 32 * hh, 0.f, 0.f, p.scale_log2, 32 * hh, cmin,
+                              TS, pp, pds);
       // the packed columns overlap only this warp's own, already loaded fp32 columns
       tmem_st16(tmem + lane_off + col_s(b) + 32 * hh, pp);
       tmem_st16(tmem + lane_off + col_dp(b) + 32 * hh, pds);
@@ -576,7 +589,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld32(tmem + lane_off + col_s(b) + 32 * hh, sv);
       tmem_ld32(tmem + lane_off + col_dp(b) + 32 * hh, dpv);
       tmem_wait_ld();
-      p_ds_chunk(sv, dpv, nullptr, nullptr, row_lse2, row_delta, false, p.scale_log2, 32 * hh, 0, cut, pp, pds);
+      p_ds_chunk_packed<false>(sv, dpv, nullptr, nullptr, row_lse2, row_delta, p.scale_log2, 32 * hh, 0, cut, pp,
+                               pds);
       tmem_st16(tmem + lane_off + col_s(b) + 32 * hh, pds);  // only dS feeds the dQ MMA
       tmem_wait_st();
       tc_fence_before();

@@ -59,10 +59,7 @@ constexpr int kMmaWarp = 9;
 #define RING_ATTN_EMU_PAIRS_PER8 1
 #endif
 constexpr int kEmuPairsPer8 = RING_ATTN_EMU_PAIRS_PER8;
-#ifndef RING_ATTN_SPEC_EXP
-#define RING_ATTN_SPEC_EXP 1
-#endif
-constexpr float kSpecMaxSum = 1048576.0f;  // 2^20
+constexpr float kSpecMaxSum = 1048576.0f;  // 2^20: the speculative exponentials' row-sum limit
 #ifndef RING_ATTN_MMA_SPIN
 #define RING_ATTN_MMA_SPIN 0
 #endif
@@ -329,7 +326,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int c = 0; c < BN / 2; ++c) pk[c] = 0u;
       } else {
         float lb = 0.f;
-#if RING_ATTN_SPEC_EXP
         // Exponentials against the current reference maximum first. The reference moves
         // only when a block's scores rise well above it, and O/l and lse do not depend on
         // it, so a block whose row sums stay <= kSpecMaxSum (every P <= 2^20, finite) is
@@ -346,9 +342,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
           tmem_wait_ld();
           mask_scores<BN>(sr, cut);
-#else
-        {
-#endif
           const float mblk = raw_rowmax<BN>(sr) * p.scale_log2;
           float alpha = 1.f;
           bool resc = false;

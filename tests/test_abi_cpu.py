@@ -134,14 +134,29 @@ def unit_table(Bz, Hq, Hkv, S, P, causal, layout, tq=256):
 @pytest.mark.parametrize("cfg", [(1, 8, 8, 16384, 8, 1, 0), (1, 8, 8, 16384, 8, 1, 1), (2, 32, 8, 131072, 16, 1, 1),
                                  (1, 2, 2, 1024, 4, 0, 0), (1, 4, 1, 4096, 4, 1, 0), (1, 8, 8, 1 << 20, 32, 1, 1),
                                  (1, 8, 8, 16384, 8, 1, 2), (2, 8, 2, 65536, 16, 1, 2), (1, 8, 8, 1 << 20, 32, 1, 2)])
-def test_units_cover_each_block_once_longest_first(lib, cfg):
+def test_units_cover_each_block_once_in_launch_order(lib, cfg):
     Bz, Hq, Hkv, S, P, causal, layout = cfg
     tab = unit_table(Bz, Hq, Hkv, S, P, causal, layout)
     keys = {tuple(r[:4]) for r in tab}
     nblk = (S // P + 255) // 256
     assert len(keys) == len(tab) == Bz * Hq * P * nblk
     cost = tab[:, 4]
-    assert (np.diff(cost) <= 0).all(), "units must be launched longest first"
+    if causal and layout == 0:
+        assert (np.diff(cost) <= 0).all(), "units must be launched longest first"
+    else:
+        # striped or zigzag causal, non-causal: consecutive groups of nblk * (Hq/Hkv) units
+        # share (b, kv head, query shard) and run their blocks longest first
+        rep = Hq // Hkv
+        per = nblk * rep
+        groups = set()
+        for r in range(0, len(tab), per):
+            grp = tab[r:r + per]
+            key = {(x[0], x[1] // rep, x[2]) for x in grp}
+            assert len(key) == 1
+            groups |= key
+            assert (np.diff(grp[:, 4]) <= 0).all(), "blocks of a group must run longest first"
+            assert sorted(grp[:, 3].tolist()) == sorted(list(range(nblk)) * rep)
+        assert len(groups) == Bz * Hkv * P
 
 
 def test_gqa_group_members_are_adjacent_in_launch_order(lib):

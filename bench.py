@@ -2,6 +2,7 @@
 """Throughput of exact ring attention on B200: causal-adjusted TFLOP/s, one JSON line.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+                    [--pass fwd|bwd|decode|merge] [--algo auto|tcgen05|tcgen05_1sm|simt]
 
 A step is one ring_attn_fwd call over the whole workload (every query shard folds
 every KV shard in ring order). Default workload: bf16, B=1, H=8, S=1,048,576,

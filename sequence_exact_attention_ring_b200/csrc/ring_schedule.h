@@ -111,15 +111,21 @@ RA_HD int kv_tiles_for(const RingGeom& g, int i, int j, int64_t a_hi, int TK) {
 // ring steps [s_begin, s_end). A grid runs its units roughly in index order:
 //   contiguous causal: cost grows with i*nkt + (rows of tb), so units are numbered
 //     longest first by the combined index c = i*nblk + tb, descending;
-//   otherwise (striped or zigzag causal, non-causal): units are grouped by (b, kv head,
-//     query shard i); inside a group the blocks run longest first (tb descending: a
-//     block's cost grows with its local index in these layouts), with the query heads
-//     of a GQA group innermost. The units of a group walk the same ring sequence of KV
-//     shards and start together, so they meet the same K/V tiles at about the same time
-//     and L2 serves most of the re-reads. On the 1M-token causal workloads this halves
-//     the DRAM traffic of a block-major order; the power it frees raises the clock
-//     under the power cap (striped +4 %, zigzag +6 % against its exact longest-first
-//     chunk order).
+//   long sequences (grouped_order: one (b, kv head)'s K and V take >= 32 MiB in
+//     bf16, so the K/V of the heads in flight no longer fits in L2), striped, zigzag
+//     or non-causal: units are grouped by (b, kv head, query shard i); inside a group
+//     the blocks run longest first (tb descending: a block's cost grows with its local
+//     index in these layouts), with the query heads of a GQA group innermost. The
+//     units of a group walk the same ring sequence of KV shards and start together, so
+//     they meet the same K/V tiles at about the same time and L2 serves most of the
+//     re-reads. On the 1M-token causal workloads this halves the DRAM traffic of the
+//     block-major order below; the power it frees raises the clock under the power cap
+//     (striped +4 %, zigzag +6 %);
+//   shorter sequences: longest first over the whole grid, which matters when the grid
+//     is a few waves deep; zigzag causal with whole blocks per chunk walks the 2P
+//     chunks from the last to the first (cost grows with the block's global position);
+//     striped causal and non-causal order by tb descending, inside a tb by (b, kv
+//     head, i, head in the GQA group).
 struct Unit {
   int b, h, i, tb;
 };
@@ -130,6 +136,10 @@ RA_HD int64_t num_units(const RingGeom& g, int BQ, int q_shard_only) {
   int64_t shards = q_shard_only >= 0 ? 1 : g.P;
   return (int64_t)g.B * g.Hq * shards * num_row_blocks(g, BQ);
 }
+
+// K and V of one (b, kv head) take 4*S*D bytes in bf16; at >= 32 MiB the grouped
+// launch orders are used (see above).
+RA_HD bool grouped_order(const RingGeom& g) { return g.S * (int64_t)g.D >= ((int64_t)1 << 23); }
 
 RA_HD Unit decode_unit(const RingGeom& g, int BQ, int q_shard_only, int64_t u) {
   const int64_t nblk = num_row_blocks(g, BQ);
@@ -156,11 +166,37 @@ RA_HD Unit decode_unit(const RingGeom& g, int BQ, int q_shard_only, int64_t u) {
     r.h = (int)((bg % g.Hkv) * rep + bh % rep);
     return r;
   }
-  int64_t x = u;  // (((b*Hkv + kvh)*P + i)*nblk + (nblk-1-tb))*rep + hr
+  if (grouped_order(g)) {
+    int64_t x = u;  // (((b*Hkv + kvh)*P + i)*nblk + (nblk-1-tb))*rep + hr
+    const int hr = (int)(x % rep);
+    x /= rep;
+    r.tb = (int)(nblk - 1 - x % nblk);
+    x /= nblk;
+    r.i = (int)(x % g.P);
+    x /= g.P;
+    const int kvh = (int)(x % g.Hkv);
+    r.b = (int)(x / g.Hkv);
+    r.h = kvh * rep + hr;
+    return r;
+  }
+  if (g.causal && g.layout == kZigzag && (g.Sq / 2) % BQ == 0) {
+    const int64_t bh_n = (int64_t)g.B * g.Hq;
+    const int64_t nbc = nblk / 2;  // blocks per chunk
+    const int64_t pos = (int64_t)g.P * nblk - 1 - u / bh_n;
+    const int c = (int)(pos / nbc);
+    r.i = c < g.P ? c : 2 * g.P - 1 - c;
+    r.tb = (int)((c < g.P ? 0 : nbc) + pos % nbc);
+    int64_t bh = u % bh_n;
+    int64_t bg = bh / rep;
+    r.b = (int)(bg / g.Hkv);
+    r.h = (int)((bg % g.Hkv) * rep + bh % rep);
+    return r;
+  }
+  const int64_t per_tb = (int64_t)g.B * g.Hq * g.P;
+  r.tb = (int)(nblk - 1 - u / per_tb);
+  int64_t x = u % per_tb;  // ((b*Hkv + kvh)*P + i)*rep + hr
   const int hr = (int)(x % rep);
   x /= rep;
-  r.tb = (int)(nblk - 1 - x % nblk);
-  x /= nblk;
   r.i = (int)(x % g.P);
   x /= g.P;
   const int kvh = (int)(x % g.Hkv);
@@ -249,9 +285,10 @@ RA_HD int64_t num_kv_units(const RingGeom& g, int TK) { return (int64_t)g.B * g.
 // A KV tile's work grows as its first token falls. Contiguous causal: shard j,
 // then tile (the earliest tiles of the sequence first, longest first); zigzag
 // causal with whole tiles per chunk: chunk 0..2P-1, then tile (longest first);
-// otherwise: shard j, then tile ascending, so the concurrently running tiles of
-// one shard walk the same ring sequence of query shards and share Q and dO
-// through L2. (b, kv head) is innermost.
+// otherwise, for long sequences (grouped_order): shard j, then tile ascending, so
+// the concurrently running tiles of one shard walk the same ring sequence of query
+// shards and share Q and dO through L2; for shorter ones: tile, then shard (longest
+// first). (b, kv head) is innermost.
 RA_HD KvUnit decode_kv_unit(const RingGeom& g, int TK, int64_t u) {
   const int64_t nkt = num_kv_tiles(g, TK);
   const int64_t bg_n = (int64_t)g.B * g.Hkv;
@@ -268,9 +305,12 @@ RA_HD KvUnit decode_kv_unit(const RingGeom& g, int TK, int64_t u) {
     const int c = (int)(pos / tpc);
     r.j = c < g.P ? c : 2 * g.P - 1 - c;
     r.kt = (int)((c < g.P ? 0 : tpc) + pos % tpc);
-  } else {
+  } else if (grouped_order(g)) {
     r.j = (int)(pos / nkt);
     r.kt = (int)(pos % nkt);
+  } else {
+    r.kt = (int)(pos / g.P);
+    r.j = (int)(pos % g.P);
   }
   return r;
 }

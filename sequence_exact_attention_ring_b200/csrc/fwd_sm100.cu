@@ -34,8 +34,10 @@
 //   * exponentials are base 2 with log2(e) folded into the scale;
 //   * the running maximum used for the exponent is only moved when the block
 //     maximum exceeds it by more than 8 (log2 units); then O and l are rescaled.
-//     Otherwise exponents stay <= 2^8, exact in fp32 and bf16 range. The final O/l
-//     and lse are invariant to the reference maximum;
+//     A block is first exponentiated against the current maximum and kept when its
+//     row sums stay <= 2^20 (every P <= 2^20, finite); otherwise, and for a row's
+//     first block, the block maximum is taken and the rule above applies. The
+//     final O/l and lse are invariant to the reference maximum;
 //   * P is rounded to bf16 before P V (as the listing does with `.to(v.dtype)`),
 //     l sums the unrounded fp32 P.
 #include <cuda.h>

@@ -6,7 +6,9 @@
 // section 3: m_new = max(m_old, rowmax S), alpha = exp(m_old - m_new),
 // P = exp(S - m_new), l = l*alpha + rowsum P, O = O*alpha + P V, in base 2 with
 // scale*log2(e) folded in, and with the reference maximum moved only when the
-// block maximum exceeds it by more than kRescaleLog2 (so exponents stay <= 2^8).
+// block maximum exceeds it by more than kRescaleLog2. The tensor-core kernels first
+// exponentiate a block against the current reference and keep the result when every
+// row sum stays <= 2^20 (finite); only then do they take the block maximum.
 #pragma once
 
 #include <math.h>

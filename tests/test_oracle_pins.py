@@ -234,6 +234,77 @@ def test_online_ring_heavy_logits_no_nan():
         np.testing.assert_allclose(L2, L1, rtol=1e-13, atol=1e-10)
 
 
+def _lazy_speculative_ring(q, k, v, P, causal, layout, scale, tile, cap=2.0 ** 20, thresh=8.0):
+    """The tensor-core kernels' block rule, restated in fp64 (a check of the rule, not
+    the oracle): base-2 exponentials against a reference maximum m that moves lazily. A
+    block is first exponentiated against the current m and kept when its row sum stays
+    <= cap; otherwise (and for a row's first visible block) the block maximum is taken, and
+    m moves to it when it exceeds m by more than thresh, rescaling l and O."""
+    B, Hq, S, D = q.shape
+    rep = Hq // k.shape[1]
+    c = scale / math.log(2.0)
+    O = np.zeros(q.shape)
+    L = np.full(q.shape[:3], -np.inf)
+    with np.errstate(over="ignore", invalid="ignore"):
+        for b in range(B):
+            for h in range(Hq):
+                g = h // rep
+                for i in range(P):
+                    tq = oracle.shard_tokens(S, P, layout, i)
+                    m = np.full(len(tq), -np.inf)
+                    l = np.zeros(len(tq))
+                    o = np.zeros((len(tq), D))
+                    for s in range(P):
+                        tk = oracle.shard_tokens(S, P, layout, (i - s) % P)
+                        for kb in range(0, len(tk), tile):
+                            tkb = tk[kb:kb + tile]
+                            x = (q[b, h, tq] @ k[b, g, tkb].T) * c
+                            x[~oracle.block_allowed(tq, tkb, causal)] = -np.inf
+                            p = np.exp2(x - np.where(np.isfinite(m), m, 0.0)[:, None])
+                            keep = np.isfinite(m) & (p.sum(1) <= cap)
+                            mb = x.max(1)
+                            move = ~keep & (mb > m + thresh)
+                            alpha = np.where(np.isfinite(m), np.exp2(m - mb), 0.0)
+                            l = np.where(move, l * alpha, l)
+                            o = np.where(move[:, None], o * alpha[:, None], o)
+                            m = np.where(move, mb, m)
+                            redo = np.exp2(x - np.where(np.isfinite(m), m, 0.0)[:, None])
+                            p = np.where(keep[:, None], p, redo)
+                            l = l + p.sum(1)
+                            o = o + p @ v[b, g, tkb]
+                    O[b, h, tq] = o / l[:, None]
+                    L[b, h, tq] = (m + np.log2(l)) * math.log(2.0)
+    return O, L
+
+
+@pytest.mark.parametrize("layout", ["contiguous", "striped", "zigzag"])
+@pytest.mark.parametrize("pattern", ["plain", "rising", "jump"])
+@pytest.mark.parametrize("cap", [2.0 ** 20, 1.0])
+def test_lazy_speculative_reference_maximum_equals_full_softmax(layout, pattern, cap):
+    """O/l and lse do not depend on the reference maximum the exponentials use, as long as
+    nothing overflows: the kernels' speculative block rule equals full softmax (cap = 1
+    forces the exact-maximum path on almost every block)."""
+    q, k, v = qkv(1, 2, 2, 64, 8, seed=91)
+    if pattern == "rising":
+        k = k * (1.0 + 6.0 * np.arange(64) / 64.0)[None, None, :, None]
+    elif pattern == "jump":
+        k[:, :, [5, 23, 40]] *= 400.0
+    O1, L1 = oracle.attention_reference(q, k, v, True, 0.5)
+    O2, L2 = _lazy_speculative_ring(q, k, v, 4, True, layout, 0.5, tile=4, cap=cap)
+    assert np.isfinite(O2).all() and np.isfinite(L2).all()
+    np.testing.assert_allclose(O2, O1, atol=1e-11, rtol=0)
+    np.testing.assert_allclose(L2, L1, rtol=1e-12, atol=1e-11)
+
+
+def test_speculative_rule_needs_a_finite_cap():
+    """Accepting every speculative block (no cap) lets a score far above the reference
+    overflow: the sum check is what keeps the rule exact."""
+    q, k, v = qkv(1, 2, 2, 64, 8, seed=91)
+    k[:, :, [5, 23, 40]] *= 400.0
+    O2, L2 = _lazy_speculative_ring(q, k, v, 4, True, "striped", 0.5, tile=4, cap=np.inf)
+    assert not (np.isfinite(O2).all() and np.isfinite(L2).all())
+
+
 # ---------------------------------------------------------------- merge
 
 def _partition_partials(q, k, v, causal, scale, labels, n_parts):

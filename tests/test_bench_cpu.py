@@ -93,3 +93,21 @@ def test_clock_sampler_parses_reasons():
     s.proc = FakeProc()
     d = s.stop()
     assert d["sm_mhz"] == 1800 and d["sm_max_mhz"] == 1965 and d["reasons"] == ["sw_power_cap"]
+
+
+def test_traffic_figure_only_for_the_measured_kernel_source(tmp_path, monkeypatch):
+    """roofline.traffic comes from the committed ncu figure only while the kernel sources
+    hash to the value recorded with it; any source change makes it null."""
+    sys.path.insert(0, ROOT)
+    import bench
+    f = tmp_path / "traffic.json"
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(f))
+    f.write_text(json.dumps({"kernel_source_sha256": bench.kernel_source_sha256(),
+                             "bytes_per_launch": {"c5_bf16_s1m_striped": 123.0}}))
+    assert bench.kernel_traffic_per_launch("c5_bf16_s1m_striped") == 123.0
+    assert bench.kernel_traffic_per_launch("c4_bf16_gqa_s128k") is None
+    f.write_text(json.dumps({"kernel_source_sha256": "0" * 64, "bytes_per_launch": {"c5_bf16_s1m_striped": 123.0}}))
+    assert bench.kernel_traffic_per_launch("c5_bf16_s1m_striped") is None
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(tmp_path / "missing.json"))
+    assert bench.kernel_traffic_per_launch("c5_bf16_s1m_striped") is None
+

@@ -58,10 +58,6 @@ constexpr int BN = 128;          // keys per KV tile
 constexpr int NQ = 2;            // query tiles per CTA
 constexpr int BQ = BM * NQ;      // query rows per unit
 constexpr int kSmemLimit = 232448;  // 227 KiB of dynamic shared memory per CTA
-#ifndef RING_ATTN_PREFETCH_TILES
-#define RING_ATTN_PREFETCH_TILES 0
-#endif
-constexpr int kPrefetchTiles = RING_ATTN_PREFETCH_TILES;  // K/V tiles prefetched into L2 ahead of the ring
 constexpr int BOXW = 64;         // bf16 elements per TMA box row (128 bytes, 128B swizzle)
 constexpr int kThreads = 384;
 constexpr int kLaunchRegs = 168;     // 65536 / 384 rounded down to a multiple of 8
@@ -69,18 +65,13 @@ constexpr int kRegsSoftmax = 208;    // per thread, warpgroups 0 and 1
 constexpr int kRegsOther = 88;       // per thread, warpgroup 2
 static_assert(2 * kRegsSoftmax + kRegsOther <= 3 * kLaunchRegs, "register split exceeds the launch pool");
 constexpr int kProducerWarp = 8;
-#ifndef RING_ATTN_PRODUCER_SLEEP_NS
-#define RING_ATTN_PRODUCER_SLEEP_NS 64
-#endif
-constexpr uint32_t kProducerSleepNs = RING_ATTN_PRODUCER_SLEEP_NS;  // the producer polls slots this often
+constexpr uint32_t kProducerSleepNs = 64;  // the producer polls slots this often (other back-offs measured neutral)
 constexpr int kMmaWarp = 9;
 // Of every 8 column pairs of a score row, this many take 2^x from the FMA-pipe
 // polynomial (exp2_poly2) and the rest from the MUFU ex2 unit, which the tensor
 // cores would otherwise wait on (both run at 16 results/clock/SM for this shape).
-#ifndef RING_ATTN_EMU_PAIRS_PER8
-#define RING_ATTN_EMU_PAIRS_PER8 0
-#endif
-constexpr int kEmuPairsPer8 = RING_ATTN_EMU_PAIRS_PER8;
+// At D = 64 the share did not pay (576-588 against 591 TFLOP/s), so it is 0 here.
+constexpr int kEmuPairsPer8 = 0;
 constexpr float kSpecMaxSum = 1048576.0f;  // 2^20: the speculative exponentials' row-sum limit
 
 template <int D>
@@ -201,19 +192,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      TileWalk w = walk_begin(g, U.i, a_hi, BN, p.s_begin, p.s_end);
-      TileWalk wp = w;  // L2 prefetch cursor, kPrefetchTiles ahead of w
-      for (int t = 0; t < kPrefetchTiles && walk_valid(wp); ++t) walk_next(g, wp, a_hi, BN);
-      for (; walk_valid(w); walk_next(g, w, a_hi, BN)) {
-        if (kPrefetchTiles > 0 && walk_valid(wp)) {
-          int p1, p2;
-          shard_map_coords(g, wp.j, wp.kb * BN, p1, p2);
-          for (int bx = 0; bx < C::kBoxes; ++bx) {
-            tma_prefetch_l2_4d(&tm_k, bx * BOXW, p1, p2, bh_kv);
-            tma_prefetch_l2_4d(&tm_v, bx * BOXW, p1, p2, bh_kv);
-          }
-          walk_next(g, wp, a_hi, BN);
-        }
+      for (TileWalk w = walk_begin(g, U.i, a_hi, BN, p.s_begin, p.s_end); walk_valid(w);
+           walk_next(g, w, a_hi, BN)) {
         int c1, c2;
         shard_map_coords(g, w.j, w.kb * BN, c1, c2);
         for (int kv = 0; kv < 2 && ok; ++kv, ++n) {

@@ -45,28 +45,16 @@ constexpr int kRegsSoftmax = 208;
 constexpr int kRegsOther = 88;
 static_assert(2 * kRegsSoftmax + kRegsOther <= 3 * kLaunchRegs, "register split exceeds the launch pool");
 constexpr int kProducerWarp = 8;
-#ifndef RING_ATTN_PRODUCER_SLEEP_NS
-#define RING_ATTN_PRODUCER_SLEEP_NS 64
-#endif
-constexpr uint32_t kProducerSleepNs = RING_ATTN_PRODUCER_SLEEP_NS;  // the producer polls slots this often
+constexpr uint64_t kCopyGraceNs = 2000000;  // after a watchdog abort, see the producer
+constexpr uint32_t kProducerSleepNs = 64;  // the producer polls slots this often (other back-offs measured neutral)
 constexpr int kMmaWarp = 9;
 // Of every 8 column pairs of a score row, this many take 2^x from the FMA-pipe
 // polynomial (exp2_poly2) and the rest from the MUFU ex2 unit (the exponentials are
 // evaluated in phases, exp_pack_phased). On the 1M-token causal workload, with the
 // speculative exponentials below: 1 of 8 measured 1015 TFLOP/s, 2 of 8 1003, 3 of 8 988,
 // 4 of 8 938 (one box, 1462 MHz).
-#ifndef RING_ATTN_EMU_PAIRS_PER8
-#define RING_ATTN_EMU_PAIRS_PER8 1
-#endif
-constexpr int kEmuPairsPer8 = RING_ATTN_EMU_PAIRS_PER8;
+constexpr int kEmuPairsPer8 = 1;
 constexpr float kSpecMaxSum = 1048576.0f;  // 2^20: the speculative exponentials' row-sum limit
-#ifndef RING_ATTN_MMA_SPIN
-#define RING_ATTN_MMA_SPIN 0
-#endif
-// The MMA issuer's P-ready waits: 1 = poll without suspending.
-__device__ __forceinline__ bool wait_p_ready(uint64_t* bar, uint32_t parity, const Watchdog& wd) {
-  return RING_ATTN_MMA_SPIN ? mbar_wait_spin(bar, parity, wd) : mbar_wait_cluster(bar, parity, wd);
-}
 constexpr uint16_t kPairMask = 0x3;
 
 constexpr int kSmemLimit = 232448;
@@ -205,11 +193,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
       }
       if (!ok && any) {
-        // wind down: this CTA's own copies must land before its shared memory goes away;
-        // their bytes are counted on the leader's barriers, so give them a fixed grace
-        // period instead of a barrier wait
+        // wind down: this CTA's own copies must land before its shared memory goes away.
+        // Their bytes are counted on the leader's barriers, and mbarrier waits take only
+        // barriers of the waiting CTA, so the producer gives them a fixed grace period
+        // (a 16 KiB tile copy completes in microseconds; the grace is about 1000 times that).
         const uint64_t t0 = global_timer_ns();
-        while (global_timer_ns() - t0 < 2000000ull) {
+        while (global_timer_ns() - t0 < kCopyGraceNs) {
         }
       }
     } else if (warp == kMmaWarp && leader) {
@@ -263,7 +252,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (int64_t n = 0; ok && n < N; ++n) {
         const bool more = n + 1 < N;
         if (!(ok = wait_all(mbar_wait_cluster(&full[vslot(n)], vphase(n), wd)))) break;
-        if (!(ok = wait_all(wait_p_ready(&bars[kPReady + 0], (uint32_t)(n & 1), wd)))) break;
+        if (!(ok = wait_all(mbar_wait_cluster(&bars[kPReady + 0], (uint32_t)(n & 1), wd)))) break;
         tc_fence_after();
         issue_pv(0, vslot(n), n == 0);
         if (more) {
@@ -274,7 +263,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         } else {
           commit(&bars[kODone + 0]);
         }
-        if (!(ok = wait_all(wait_p_ready(&bars[kPReady + 1], (uint32_t)(n & 1), wd)))) break;
+        if (!(ok = wait_all(mbar_wait_cluster(&bars[kPReady + 1], (uint32_t)(n & 1), wd)))) break;
         tc_fence_after();
         issue_pv(1, vslot(n), n == 0);
         commit(&empty[vslot(n)]);

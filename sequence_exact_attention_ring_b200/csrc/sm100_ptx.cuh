@@ -58,33 +58,17 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
-// How a waiting thread polls an mbarrier: 0 = try_wait (the hardware may suspend
-// the thread for a system-defined time), 1 = test_wait (never suspends),
-// 2 = try_wait with an explicit suspend-time hint of RING_ATTN_WAIT_HINT_NS.
-#ifndef RING_ATTN_WAIT_MODE
-#define RING_ATTN_WAIT_MODE 0
-#endif
-#ifndef RING_ATTN_WAIT_HINT_NS
-#define RING_ATTN_WAIT_HINT_NS 100
-#endif
-#if RING_ATTN_WAIT_MODE == 1
-#define RA_MBAR_POLL(sem) "mbarrier.test_wait.parity" sem ".shared::cta.b64 p, [%1], %2;\n\t"
-#define RA_MBAR_HINT
-#elif RING_ATTN_WAIT_MODE == 2
-#define RA_MBAR_POLL(sem) "mbarrier.try_wait.parity" sem ".shared::cta.b64 p, [%1], %2, %3;\n\t"
-#define RA_MBAR_HINT , "n"(RING_ATTN_WAIT_HINT_NS)
-#else
-#define RA_MBAR_POLL(sem) "mbarrier.try_wait.parity" sem ".shared::cta.b64 p, [%1], %2;\n\t"
-#define RA_MBAR_HINT
-#endif
-
+// Waiting threads poll with mbarrier.try_wait (the hardware may suspend the thread
+// for a system-defined time between checks). Measured against test_wait (never
+// suspends) and try_wait with a 20-100 ns suspend hint, it was 0-3 % faster.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{\n\t.reg .pred p;\n\t" RA_MBAR_POLL("")
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity) RA_MBAR_HINT
+      : "r"(smem_u32(bar)), "r"(parity)
       : "memory");
   return ok != 0;
 }
@@ -124,41 +108,20 @@ __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// Memory-ordering qualifiers of the pair barriers that other CTAs signal:
-// 0 = release/acquire at cluster scope, 1 = the instructions' defaults (CTA
-// scope), 2 = relaxed cluster-scope arrive with a CTA-scope acquire. The default
-// is 1: the data handed over is tensor memory, ordered by tcgen05.fence
-// before/after_thread_sync around the barrier, the same pairing used for
-// consumer releases of 2-SM MMA pipelines; the cluster-scope release/acquire
-// pair costs about 0.9 us per hand-over on B200.
-#ifndef RING_ATTN_CLUSTER_SEM
-#define RING_ATTN_CLUSTER_SEM 1
-#endif
-#if RING_ATTN_CLUSTER_SEM == 1
-#define RA_ARRIVE_SEM ""
-#define RA_WAIT_SEM ""
-#elif RING_ATTN_CLUSTER_SEM == 2
-#define RA_ARRIVE_SEM ".relaxed.cluster"
-#define RA_WAIT_SEM ""
-#else
-#define RA_ARRIVE_SEM ".release.cluster"
-#define RA_WAIT_SEM ".acquire.cluster"
-#endif
-
+// Barriers that the other CTA of a pair signals use the instructions' default
+// (CTA-scope) ordering. The data handed over is tensor memory, ordered by
+// tcgen05.fence before/after_thread_sync around the barrier, the same pairing used
+// for consumer releases of 2-SM MMA pipelines; a cluster-scope release/acquire pair
+// cost about 0.9 us per hand-over on B200.
 // Arrive on an mbarrier that may live in another CTA of the cluster.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive" RA_ARRIVE_SEM ".shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
+// Poll of a barrier that the other CTA of the pair also signals (same instruction,
+// CTA-scope ordering, see above).
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t" RA_MBAR_POLL(RA_WAIT_SEM)
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity) RA_MBAR_HINT
-      : "memory");
-  return ok != 0;
+  return mbar_try_wait(bar, parity);
 }
 
 // Bounded wait that sleeps `sleep_ns` between polls: for waiters off the critical
@@ -181,37 +144,7 @@ __device__ __forceinline__ bool mbar_wait_backoff(uint64_t* bar, uint32_t parity
   }
 }
 
-// Bounded wait that never suspends the thread (mbarrier.test_wait): for a single
-// thread on the critical path whose wake-up latency matters more than the issue
-// slots its polling takes from other warps.
-__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, const Watchdog& wd) {
-  if (mbar_test_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  while (true) {
-#pragma unroll 1
-    for (int r = 0; r < 64; ++r)
-      if (mbar_test_wait(bar, parity)) return true;
-    if (watchdog_aborted(wd)) return false;
-    if (global_timer_ns() - t0 > wd.limit_ns) {
-      watchdog_trip(wd);
-      return false;
-    }
-  }
-}
-
-// Bounded wait with cluster-scope acquire (for barriers other CTAs of the pair signal).
+// Bounded wait on a barrier that the other CTA of the pair also signals.
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, const Watchdog& wd) {
   if (mbar_try_wait_cluster(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
@@ -247,14 +180,6 @@ __device__ __forceinline__ void tma_load_4d(void* smem_dst, const void* tmap, ui
       " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(smem_dst)),
       "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
       : "memory");
-}
-
-// Prefetch a 4-D tile into L2 only (no shared memory, no completion signal).
-__device__ __forceinline__ void tma_prefetch_l2_4d(const void* tmap, int c0, int c1, int c2, int c3) {
-  asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
-                   reinterpret_cast<uint64_t>(tmap)),
-               "r"(c0), "r"(c1), "r"(c2), "r"(c3)
-               : "memory");
 }
 
 // 2-SM form: data lands in this CTA's shared memory, completion bytes are counted

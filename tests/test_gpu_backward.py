@@ -122,3 +122,57 @@ def test_backward_cuda_core_path(cuda_lib, case):
             assert np.abs(g - r).max() <= 1e-4 * np.abs(r).max(), f"{case} {name}"
         else:
             assert_grad(got, r, f"{case} {name}")
+
+
+# ------------------------------------------------------------------ long sequences
+# From S*D >= 2^23 (S >= 65536 at D = 128) the dK/dV and dQ kernels switch to their
+# grouped launch orders, the regime the backward benchmark runs. Every element of
+# dq, dk and dv is compared with the fp64 oracle at 64k tokens, for the three layouts.
+
+LONG_CASES = [
+    # (B, Hq, Hkv, S, D, P, causal, layout)
+    (1, 1, 1, 65536, 128, 8, True, "contiguous"),
+    (1, 1, 1, 65536, 128, 8, True, "striped"),
+    (1, 1, 1, 65536, 128, 8, True, "zigzag"),   # C = 4096: whole 128-row tiles
+]
+
+
+@pytest.mark.parametrize("case", LONG_CASES, ids=lambda c: f"{c[7]}-S{c[3]}")
+def test_backward_64k_all_elements(cuda_lib, case):
+    w, q, k, v, dout, out, lse = make(*case, seed=241)
+    dq, dk, dv = ring_attention_backward(q, k, v, out, lse, dout, w.P, w.causal, w.layout, w.scale)
+    torch.cuda.synchronize()
+    ref = oracle.attention_backward_reference(q.cpu(), k.cpu(), v.cpu(), dout.cpu(), w.causal, w.scale)
+    for name, got, r in zip(("dq", "dk", "dv"), (dq, dk, dv), ref):
+        assert_grad(got, r, f"{case} {name}")
+
+
+def test_backward_c4_gqa_heavy_keys_sampled(cuda_lib):
+    """The 131k GQA workload with heavy keys (striped, P = 16, 4 query heads per kv head):
+    1024 seeded dQ rows plus the shard-boundary rows; dK/dV of the last 64 tokens of
+    every (batch, kv head), which hold the last key of every shard; column sums over all keys."""
+    w = synthetic.get("c4_bf16_gqa_s128k")
+    q, k, v = synthetic.make_inputs(w, "cuda")
+    dout = synthetic.make_dout(w, "cuda")
+    out, lse = ring_attention(q, k, v, w.P, w.causal, w.layout, w.scale)
+    dq, dk, dv = ring_attention_backward(q, k, v, out, lse, dout, w.P, w.causal, w.layout, w.scale)
+    torch.cuda.synchronize()
+    qh, kh, vh, doh = q.cpu(), k.cpu(), v.cpu(), dout.cpu()
+    rows = synthetic.sample_rows(w, 1024)
+    ref_q = oracle.backward_rows_dq(qh, kh, vh, doh, rows, w.causal, w.scale)
+    got_q = torch.stack([dq[b, h, t] for b, h, t in rows])
+    assert_grad(got_q, ref_q, "c4 dq rows")
+    keys = [(b, g, u) for b in range(w.B) for g in range(w.Hkv) for u in range(w.S - 64, w.S)]
+    ref_k, ref_v = oracle.backward_rows_dkdv(qh, kh, vh, doh, keys, w.causal, w.scale)
+    got_k = torch.stack([dk[b, g, u] for b, g, u in keys])
+    got_v = torch.stack([dv[b, g, u] for b, g, u in keys])
+    assert_grad(got_k, ref_k, "c4 dk last keys")
+    assert_grad(got_v, ref_v, "c4 dv last keys")
+    # every row of P sums to 1 and every row of dS to 0, per kv head over its query heads:
+    # sum_u dV_u = sum over the group's rows of dO_t, and sum_u dK_u = 0
+    rep = w.Hq // w.Hkv
+    sv = dv.double().sum(dim=2)
+    so = dout.double().view(w.B, w.Hkv, rep, w.S, w.D).sum(dim=(2, 3))
+    assert (sv - so).abs().max().item() <= 2e-2 * dv.double().abs().sum(dim=2).max().item()
+    sk = dk.double().sum(dim=2)
+    assert sk.abs().max().item() <= 2e-2 * dk.double().abs().sum(dim=2).max().item()

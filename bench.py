@@ -2,14 +2,20 @@
 """Throughput of exact ring attention on B200: causal-adjusted TFLOP/s, one JSON line.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
-                    [--pass fwd|bwd|decode|merge] [--algo auto|tcgen05|tcgen05_1sm|simt]
+                    [--pass fwd|bwd|decode|merge|ring] [--algo auto|tcgen05|tcgen05_1sm|simt]
+                    [--ring-ranks R]
 
 A step is one ring_attn_fwd call over the whole workload (every query shard folds
 every KV shard in ring order). Default workload: bf16, B=1, H=8, S=1,048,576,
 D=128, P=32, causal striped. Inputs are seeded synthetic tensors resident in HBM
-(larger than L2, so no flush is needed between steps). With N>1 (torchrun) every
-rank runs its own independent instance (seed + rank): weak scaling, no collective
-on the data path; the step time is the max over ranks.
+(larger than L2, so no flush is needed between steps). With N>1 every rank runs
+its own independent instance (seed + rank): weak scaling, no collective on the data
+path; the step time is the max over ranks. `--gpus N` outside torchrun starts the N
+ranks itself.
+
+--pass ring spreads one sequence over ranks instead (the pages' ring: KV shards
+travel between ranks while each rank folds the one it holds): virtual ranks on one
+GPU, or one rank per GPU under torchrun.
 
 --impl reference times the fp64 CPU oracle (the correctness reference) on a
 bounded sample of query rows of the same workload; rank 0 only.
@@ -55,10 +61,26 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
-    ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd", "decode", "merge"],
+    ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd", "decode", "merge", "ring"],
                     help="fwd: the forward hot path (the headline line); bwd: ring_attn_bwd on the same workload; "
-                         "decode: one decode step against the workload's K/V as the cache")
+                         "decode: one decode step against the workload's K/V as the cache; ring: the ring spread "
+                         "over ranks (virtual ranks on one GPU, or one rank per GPU under torchrun)")
+    ap.add_argument("--ring-ranks", type=int, default=8,
+                    help="--pass ring on one GPU: number of virtual ranks the sequence is spread over")
     return ap.parse_args()
+
+
+def relaunch_under_torchrun(args) -> int:
+    """`--gpus N` (N > 1) outside torchrun: start N ranks on this node with torchrun and
+    return its exit code (rank 0 prints the line)."""
+    import socket
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.run(cmd).returncode
 
 
 # ------------------------------------------------------------------ distributed plumbing
@@ -73,7 +95,8 @@ def dist_setup(args):
         backend = "nccl" if torch.cuda.is_available() else "gloo"
         if torch.cuda.is_available():
             torch.cuda.set_device(local)
-        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=600))
+        # a short timeout: ranks that wait for one another end with an error, not a hang
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return world, rank, local
@@ -239,7 +262,7 @@ def run_reference(args, world, rank):
     value = statistics.median(rates)
     total = w.causal_flops()
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1,
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": total / (value * 1e12) * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -549,9 +572,125 @@ def run_merge(args, world, rank, local):
     }))
 
 
+RING_METRIC = "ring spread over ranks (forward): causal-adjusted attention TFLOP/s"
+
+
+def run_ring(args, world, rank, local):
+    """The forward ring with the sequence spread over ranks (RingAttention deep-architecture
+    article, sections 2, 4, 5): every rank keeps one query shard, the KV shards travel the
+    ring, each step is one ring_attn_fwd_ring_step launch whose epilogue folds the block
+    into the rank's running state.
+      one GPU: --ring-ranks virtual ranks, each with its own buffers and streams; the KV
+               shards move by device-to-device copies on copy streams while steps run;
+      N GPUs (torchrun): one rank per GPU, KV shards over NCCL point-to-point into the
+               GPU's own buffers.
+    The whole job is one sequence (strong scaling). Also reports the per-step copy and
+    compute durations (the zero-bubble condition of section 4) and, on one GPU, the
+    single-launch ring_attn_fwd time of the same workload."""
+    from sequence_exact_attention_ring_b200 import binding, ring, ring_attention
+    w = synthetic.get(args.workload)
+    binding.load()
+    dev = torch.device("cuda", local if world > 1 else 0)
+    R = world if world > 1 else args.ring_ranks
+    if w.S % R or (w.layout == "zigzag" and w.S % (2 * R)):
+        raise SystemExit(f"S={w.S} does not split into {R} ring shards")
+    q, k, v = synthetic.make_inputs(w, dev)
+    stream = torch.cuda.current_stream(dev)
+    fused_ms = None
+    if world == 1:
+        # the single-launch forward of the same workload, for comparison
+        out = torch.empty_like(q)
+        lse = torch.empty((w.B, w.Hq, w.S), dtype=torch.float32, device=dev)
+        ring_attention(q, k, v, w.P, w.causal, w.layout, w.scale, out=out, lse=lse, stream=stream)
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(2):
+            ring_attention(q, k, v, w.P, w.causal, w.layout, w.scale, out=out, lse=lse, stream=stream)
+        f1.record(stream)
+        torch.cuda.synchronize(dev)
+        fused_ms = f0.elapsed_time(f1) / 2
+        del out, lse
+    qs, ks, vs = (ring.split_shards(t, R, w.layout) for t in (q, k, v))
+    del q, k, v
+    if world > 1:
+        qs, ks, vs = [qs[rank]], [ks[rank]], [vs[rank]]
+    torch.cuda.synchronize(dev)
+    torch.cuda.empty_cache()
+    if world == 1:
+        vr = ring.VirtualRing(qs, ks, vs, w.causal, w.layout, w.scale)
+
+        def step(timing=False):
+            return vr.run(timing=timing)
+    else:
+        comm = torch.cuda.Stream(dev)
+
+        def step(timing=False):
+            ring.ring_attention_distributed(qs[0], ks[0], vs[0], w.causal, w.layout, w.scale, stream=stream,
+                                            comm_stream=comm)
+            return None
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    sampler = ClockSampler(dev.index)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    barrier(world)
+    elapsed = max_over_ranks(t0.elapsed_time(t1), world)
+    overlap = None
+    if world == 1:
+        # one more, instrumented pass: per rank and step, the copy and the compute durations
+        tm = step(timing=True)
+        torch.cuda.synchronize(dev)
+        comp = [[a.elapsed_time(b) for a, b in per] for per in tm["compute"]]
+        cop = [[a.elapsed_time(b) for a, b in per] for per in tm["copy"]]
+        overlap = {"virtual_ranks": R, "step_ms_wall": elapsed / args.steps,
+                   "fused_single_launch_ms": fused_ms,
+                   "compute_ms_per_rank_max": max(sum(c) for c in comp),
+                   "copy_ms_per_rank_max": max(sum(c) for c in cop) if R > 1 else 0.0,
+                   "copy_ms_per_step_max": max(max(c) for c in cop) if R > 1 else 0.0,
+                   "kv_bytes_per_step_per_rank": 2 * ks[0].numel() * ks[0].element_size()}
+    flops = w.causal_flops()
+    value = flops * args.steps / (elapsed * 1e-3) / 1e12
+    peaks, peak_src = measured_peaks()
+    peak = float(peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"])
+    skipped = 0
+    if w.causal and w.layout == "contiguous":
+        skipped = R * (R - 1) // 2  # fully masked blocks: no launch unless first or last
+    launches_per_step = R * R - skipped + (R - 1 if skipped else 0)
+    clocks_all = gather_objects(clocks, world)
+    if rank != 0:
+        return
+    print(json.dumps({
+        "metric": RING_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed / args.steps, "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": dict(workload_config(w), **{"pass": "ring", "ring_ranks": R,
+                                              "transport": "device-to-device copies between virtual ranks"
+                                              if world == 1 else "NCCL point-to-point between GPUs"}),
+        "roofline": {"bound": "tensor", "achieved": value / world, "peak": peak, "unit": "TFLOP/s",
+                     "frac": value / world / peak, "traffic": None,
+                     "peak_source": f"{peak_src} bf16_tflops_sustained",
+                     "kernel": "ring_fwd_sm100_2sm_kernel (one launch per ring step, fold epilogue)"},
+        "overlap": overlap,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks_all[0] if world == 1 else {"per_rank": clocks_all},
+    }))
+
+
 def main():
     args = parse()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(relaunch_under_torchrun(args))
     world, rank, local = dist_setup(args)
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but {world} ranks were launched")
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)
@@ -561,6 +700,8 @@ def main():
             run_decode(args, world, rank, local)
         elif args.which == "merge":
             run_merge(args, world, rank, local)
+        elif args.which == "ring":
+            run_ring(args, world, rank, local)
         else:
             run_ours(args, world, rank, local)
     finally:

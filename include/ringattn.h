@@ -117,6 +117,42 @@ int ring_attn_fwd_step(const void* q, const void* k, const void* v, float* o_par
                        void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * One step of a ring spread over devices, on shard-local buffers, folded into a
+ * running state. This is what one device of the pages' ring runs at each step
+ * (RingAttention deep-architecture article, techknowgenie, section 2 "core
+ * principle": a device keeps its query shard while KV shards pass around the ring;
+ * section 5 listing: per step the block is folded into the running (m, l, O), and the
+ * output is produced after the last step). The state between steps is kept
+ * normalised, (o, lse) with l divided out, and each step's block result is folded in
+ * with the section 3 rescale:
+ *     lse = ln(e^lse_acc + e^lse_step),  o = e^(lse_acc - lse) o_acc + e^(lse_step - lse) o_step.
+ *   q_shard   device [B, Hq,  Sq, D]  query shard q_index, rows in shard-local order
+ *   k_shard,  device [B, Hkv, Sq, D]  KV shard kv_index, shard-local order (Sq = S/P)
+ *   v_shard
+ *   o_acc     device [B, Hq, Sq, D] fp32  running state, shard-local order
+ *   lse_acc   device [B, Hq, Sq]    fp32
+ *   out       device [B, Hq, Sq, D] in dtype, written only by a LAST step
+ *   lse_out   device [B, Hq, Sq]    fp32,     written only by a LAST step
+ *   flags     RING_ATTN_STEP_FIRST: the state starts from this step (o_acc/lse_acc
+ *             are written, not read). RING_ATTN_STEP_LAST: the merged rows go to
+ *             out/lse_out and the state is left as it was. FIRST|LAST: out is this
+ *             step alone, and o_acc/lse_acc may be NULL.
+ * S, P, layout and causal describe the whole ring (shard map and causal mask on
+ * global tokens, as in ring_attn_fwd); q_index/kv_index in [0, P). Every layout
+ * runs on the tensor cores here (bf16; fp32 runs on the CUDA-core kernel). A step
+ * whose block no query row can see (contiguous causal with kv_index > q_index) and
+ * that is neither FIRST nor LAST enqueues nothing. Outputs must not alias inputs
+ * or the state. Same argument, workspace and watchdog rules as ring_attn_fwd.
+ */
+#define RING_ATTN_STEP_FIRST 1
+#define RING_ATTN_STEP_LAST 2
+int ring_attn_fwd_ring_step(const void* q_shard, const void* k_shard, const void* v_shard,
+                            float* o_acc, float* lse_acc, void* out, float* lse_out,
+                            int B, int Hq, int Hkv, int64_t S, int D, int P, int q_index, int kv_index,
+                            int causal, int layout, float scale, int dtype, int flags,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Combine n normalised partials of the same rows (the online-softmax rescale of
  * section 3 applied to states whose l is already divided out):
  *   lse = lse_max + ln sum_k exp(lse_k - lse_max),  out = sum_k exp(lse_k - lse) * o_k
@@ -203,12 +239,15 @@ int ring_attn_status(const void* workspace, void* stream);
  *   scratch_out  optional host pointer (may be NULL). On success it receives the
  *                device address of this device's scratch. Pass that address to
  *                ring_attn_status() to read the status word of the last call.
- * Setup: the first call on each device, with that device current, looks up the
- * array's device address (cudaGetSymbolAddress) and caches it. Make that first
- * call before any stream capture on that device.
- * Errors: as ring_attn_fwd. If these arguments need more workspace than the array
- * holds, it returns RING_ATTN_EWORKSPACE and enqueues nothing. If the address
- * lookup fails, it returns RING_ATTN_ECUDA.
+ * Setup: the first call in each CUDA context (the device's primary context, or a
+ * context the caller made current with the driver API) looks up the array's
+ * device address in that context (cudaGetSymbolAddress) and caches it under the
+ * context's unique id, so a context created after cudaDeviceReset gets a fresh
+ * lookup. Make that first call before any stream capture in that context.
+ * Errors: as ring_attn_fwd (the same code for the same bad argument). If these
+ * arguments need more workspace than the array holds, it returns
+ * RING_ATTN_EWORKSPACE and enqueues nothing. If the address lookup fails, it
+ * returns RING_ATTN_ECUDA.
  * Concurrency: every call on a device shares one scratch array. Calls that overlap
  * on the device (different streams, or host threads without ordering) race on the
  * status word. Order them on one stream, or use ring_attn_fwd with separate

@@ -90,6 +90,49 @@ def ring_attention_step(q, k, v, P: int, q_shard: int, kv_shard: int, causal: bo
     return o, lse
 
 
+def ring_attention_ring_step(q_shard, k_shard, v_shard, S: int, P: int, q_index: int, kv_index: int,
+                             causal: bool = True, layout="striped", scale: float | None = None, first: bool = False,
+                             last: bool = False, o_acc=None, lse_acc=None, out=None, lse_out=None, workspace=None,
+                             stream=None):
+    """One ring step on shard-local buffers (as one device of a multi-device ring runs it).
+
+    q_shard [B,Hq,Sq,D] is query shard q_index and k_shard/v_shard [B,Hkv,Sq,D] KV shard
+    kv_index, each in shard-local order. The step's block result is folded into the
+    running state o_acc [B,Hq,Sq,D] fp32 / lse_acc [B,Hq,Sq] (started on `first`); on
+    `last` the merged rows go to out (q's dtype) and lse_out. Returns (out, lse_out) on
+    a last step, else (o_acc, lse_acc). Asynchronous on `stream`.
+    """
+    _check_qkv(q_shard, k_shard, v_shard)
+    B, Hq, Sq, D = q_shard.shape
+    if Sq * P != S:
+        raise ValueError("shards must hold S / P rows")
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    dev = q_shard.device
+    if not (first and last):
+        for t, shape in ((o_acc, (B, Hq, Sq, D)), (lse_acc, (B, Hq, Sq))):
+            if t is None or tuple(t.shape) != shape or t.dtype != torch.float32 or not t.is_contiguous():
+                raise ValueError("o_acc [B,Hq,Sq,D] and lse_acc [B,Hq,Sq] must be contiguous float32 tensors")
+    if last:
+        if out is None:
+            out = torch.empty_like(q_shard)
+        if lse_out is None:
+            lse_out = torch.empty((B, Hq, Sq), dtype=torch.float32, device=dev)
+    if workspace is None:
+        wsb = _b.ring_attn_fwd_workspace_bytes(B, Hq, k_shard.shape[1], S, D, P, int(causal), _layout(layout),
+                                               _DTYPES[q_shard.dtype])
+        if wsb == 0:
+            raise _b.RingAttnError(_b.EINVAL, "ring_attn_fwd_workspace_bytes")
+        workspace = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    flags = (_b.STEP_FIRST if first else 0) | (_b.STEP_LAST if last else 0)
+    ptr = lambda t: 0 if t is None else t.data_ptr()  # noqa: E731
+    rc = _b.ring_attn_fwd_ring_step(q_shard.data_ptr(), k_shard.data_ptr(), v_shard.data_ptr(), ptr(o_acc),
+                                    ptr(lse_acc), ptr(out), ptr(lse_out), B, Hq, k_shard.shape[1], S, D, P, q_index,
+                                    kv_index, int(causal), _layout(layout), scale, _DTYPES[q_shard.dtype], flags,
+                                    workspace.data_ptr(), workspace.numel(), _stream_ptr(stream))
+    _b.check(rc, "ring_attn_fwd_ring_step")
+    return (out, lse_out) if last else (o_acc, lse_acc)
+
+
 def ring_attention_backward(q, k, v, out, lse, dout, P: int, causal: bool = True, layout="striped",
                             scale: float | None = None, workspace=None, stream=None):
     """Gradients (dq, dk, dv) of ring_attention's output against dout, from its out and lse.

@@ -29,6 +29,8 @@ ALGO_AUTO = 0
 ALGO_SIMT = 1
 ALGO_TCGEN05 = 2
 ALGO_TCGEN05_1SM = 3
+STEP_FIRST = 1
+STEP_LAST = 2
 
 _c_int, _c_i64, _c_size, _vp, _c_float = ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_float
 
@@ -44,6 +46,9 @@ SIGNATURES = {
                                     _c_int, _c_int, _c_float, _c_int, _vp, _c_size, _vp, _c_int]),
     "ring_attn_fwd_step": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_i64, _c_int, _c_int,
                                     _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _c_int, _vp, _c_size, _vp]),
+    "ring_attn_fwd_ring_step": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_i64, _c_int,
+                                         _c_int, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _c_int, _vp,
+                                         _c_size, _vp]),
     "ring_attn_merge": (_c_int, [_vp, _vp, _c_int, _c_i64, _c_int, _vp, _vp, _c_int, _vp]),
     "ring_attn_status": (_c_int, [_vp, _vp]),
     "ring_attn_bwd_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int, _c_i64, _c_int, _c_int, _c_int, _c_int,
@@ -131,6 +136,13 @@ def ring_attn_fwd_step(q, k, v, o_part, lse_part, B, Hq, Hkv, S, D, P, q_shard, 
                        dtype, algo, workspace, workspace_bytes, stream) -> int:
     return load().ring_attn_fwd_step(q, k, v, o_part, lse_part, B, Hq, Hkv, S, D, P, q_shard, kv_shard, causal,
                                      layout, scale, dtype, algo, workspace, workspace_bytes, stream)
+
+
+def ring_attn_fwd_ring_step(q_shard, k_shard, v_shard, o_acc, lse_acc, out, lse_out, B, Hq, Hkv, S, D, P, q_index,
+                            kv_index, causal, layout, scale, dtype, flags, workspace, workspace_bytes, stream) -> int:
+    return load().ring_attn_fwd_ring_step(q_shard, k_shard, v_shard, o_acc, lse_acc, out, lse_out, B, Hq, Hkv, S, D,
+                                          P, q_index, kv_index, causal, layout, scale, dtype, flags, workspace,
+                                          workspace_bytes, stream)
 
 
 def ring_attn_merge(o_parts, lse_parts, n_parts, rows, D, out, lse_out, out_dtype, stream) -> int:

@@ -91,17 +91,28 @@ int reset_status(void* workspace, cudaStream_t stream) {
 
 // Launch one ring-attention pass for the given ring-step range and output mode.
 int run_fwd(const void* q, const void* k, const void* v, void* out, float* lse, const RingGeom& g, float scale,
-            int dtype, int algo, int s_begin, int s_end, int q_shard_only, int partial, void* workspace,
+            int dtype, int algo, int s_begin, int s_end, int q_shard_only, const FwdOut& fo, void* workspace,
             cudaStream_t stream) {
   int rc = reset_status(workspace, stream);
   if (rc) return rc;
   if (algo == RING_ATTN_ALGO_TCGEN05 && g.D == 128)
-    return launch_fwd_sm100_2sm(q, k, v, out, lse, g, scale, s_begin, s_end, q_shard_only, partial,
+    return launch_fwd_sm100_2sm(q, k, v, out, lse, g, scale, s_begin, s_end, q_shard_only, fo,
                                 static_cast<int*>(workspace), watchdog_ns(), stream);
   if (algo == RING_ATTN_ALGO_TCGEN05 || algo == RING_ATTN_ALGO_TCGEN05_1SM)
-    return launch_fwd_sm100(q, k, v, out, lse, g, scale, s_begin, s_end, q_shard_only, partial,
+    return launch_fwd_sm100(q, k, v, out, lse, g, scale, s_begin, s_end, q_shard_only, fo,
                             static_cast<int*>(workspace), watchdog_ns(), stream);
-  return launch_fwd_simt(q, k, v, out, lse, g, scale, dtype, s_begin, s_end, q_shard_only, partial, stream);
+  return launch_fwd_simt(q, k, v, out, lse, g, scale, dtype, s_begin, s_end, q_shard_only, fo, stream);
+}
+
+FwdOut out_mode(int kind) {
+  FwdOut fo;
+  fo.kind = kind;
+  fo.local = 0;
+  fo.first = 0;
+  fo.last = 0;
+  fo.acc_o = nullptr;
+  fo.acc_lse = nullptr;
+  return fo;
 }
 
 }  // namespace
@@ -143,7 +154,7 @@ int ring_attn_fwd_algo(const void* q, const void* k, const void* v, void* out, f
   if (!(scale > 0.f) || !isfinite(scale)) return RING_ATTN_EINVAL;
   algo = resolve_algo(algo, dtype, g);
   if ((rc = check_algo(algo, dtype, g))) return rc;
-  return run_fwd(q, k, v, out, lse, g, scale, dtype, algo, 0, P, -1, 0, workspace,
+  return run_fwd(q, k, v, out, lse, g, scale, dtype, algo, 0, P, -1, out_mode(kOutFinal), workspace,
                  static_cast<cudaStream_t>(stream));
 }
 
@@ -169,7 +180,44 @@ int ring_attn_fwd_step(const void* q, const void* k, const void* v, float* o_par
   algo = resolve_algo(algo, dtype, g);
   if ((rc = check_algo(algo, dtype, g))) return rc;
   const int s = ring_step_of(q_shard, kv_shard, P);
-  return run_fwd(q, k, v, o_part, lse_part, g, scale, dtype, algo, s, s + 1, q_shard, 1, workspace,
+  return run_fwd(q, k, v, o_part, lse_part, g, scale, dtype, algo, s, s + 1, q_shard, out_mode(kOutPartial), workspace,
+                 static_cast<cudaStream_t>(stream));
+}
+
+int ring_attn_fwd_ring_step(const void* q_shard, const void* k_shard, const void* v_shard, float* o_acc,
+                            float* lse_acc, void* out, float* lse_out, int B, int Hq, int Hkv, int64_t S, int D,
+                            int P, int q_index, int kv_index, int causal, int layout, float scale, int dtype,
+                            int flags, void* workspace, size_t workspace_bytes, void* stream) {
+  RingGeom g;
+  int rc = check_geom(B, Hq, Hkv, S, D, P, causal, layout, dtype, &g);
+  if (rc) return rc;
+  if (q_index < 0 || q_index >= P || kv_index < 0 || kv_index >= P) return RING_ATTN_EINVAL;
+  if (flags & ~(RING_ATTN_STEP_FIRST | RING_ATTN_STEP_LAST)) return RING_ATTN_EINVAL;
+  const bool first = (flags & RING_ATTN_STEP_FIRST) != 0;
+  const bool last = (flags & RING_ATTN_STEP_LAST) != 0;
+  const bool need_acc = !(first && last);
+  if (!q_shard || !k_shard || !v_shard) return RING_ATTN_EINVAL;
+  if (need_acc && (!o_acc || !lse_acc)) return RING_ATTN_EINVAL;
+  if (last && (!out || !lse_out)) return RING_ATTN_EINVAL;
+  if (!aligned16(q_shard) || !aligned16(k_shard) || !aligned16(v_shard)) return RING_ATTN_EALIGN;
+  if (need_acc && (!aligned16(o_acc) || !aligned16(lse_acc))) return RING_ATTN_EALIGN;
+  if (last && (!aligned16(out) || !aligned16(lse_out))) return RING_ATTN_EALIGN;
+  if (!workspace || workspace_bytes < kWorkspaceHeaderBytes || !aligned16(workspace)) return RING_ATTN_EWORKSPACE;
+  if (!(scale > 0.f) || !isfinite(scale)) return RING_ATTN_EINVAL;
+  // shard-local buffers carry no chunk boundary inside a tile, so every layout tiles
+  int algo = dtype == RING_ATTN_DTYPE_BF16 ? RING_ATTN_ALGO_TCGEN05 : RING_ATTN_ALGO_SIMT;
+  if (algo == RING_ATTN_ALGO_TCGEN05 && !device_is_sm100()) return RING_ATTN_EUNSUPPORTED;
+  // a block no query row can see (contiguous causal, kv_index > q_index) adds nothing;
+  // only a first or last step still has the state to initialise or to write out
+  if (key_limit(g, q_index, kv_index, g.Sq - 1) == 0 && !first && !last) return RING_ATTN_OK;
+  FwdOut fo = out_mode(kOutFold);
+  fo.local = 1;
+  fo.first = first;
+  fo.last = last;
+  fo.acc_o = o_acc;
+  fo.acc_lse = lse_acc;
+  const int s = ring_step_of(q_index, kv_index, P);
+  return run_fwd(q_shard, k_shard, v_shard, out, lse_out, g, scale, dtype, algo, s, s + 1, q_index, fo, workspace,
                  static_cast<cudaStream_t>(stream));
 }
 
@@ -311,7 +359,8 @@ int64_t ring_attn_debug_visit_counts(int64_t S, int P, int causal, int layout, i
     const Unit U = decode_unit(g, tile_q, -1, u);
     const int64_t a0 = (int64_t)U.tb * tile_q;
     const int64_t a_hi = (a0 + tile_q - 1 < g.Sq - 1) ? a0 + tile_q - 1 : g.Sq - 1;
-    for (TileWalk w = walk_begin(g, U.i, a_hi, tile_k, 0, P); walk_valid(w); walk_next(g, w, a_hi, tile_k)) {
+    for (TileWalk w = walk_begin(g, U.i, a_hi, tile_k, 0, P); walk_valid(w);
+         walk_next(g, w, a_hi, tile_k)) {
       ++tiles;
       for (int64_t a = a0; a < a0 + tile_q && a < g.Sq; ++a) {
         const int64_t lim = key_limit(g, U.i, w.j, a);
@@ -357,7 +406,8 @@ int64_t ring_attn_debug_unit_walk(int B, int Hq, int Hkv, int64_t S, int P, int 
   const int64_t a0 = (int64_t)U.tb * tile_q;
   const int64_t a_hi = (a0 + tile_q - 1 < g.Sq - 1) ? a0 + tile_q - 1 : g.Sq - 1;
   int64_t n = 0;
-  for (TileWalk w = walk_begin(g, U.i, a_hi, tile_k, 0, P); walk_valid(w); walk_next(g, w, a_hi, tile_k), ++n) {
+  for (TileWalk w = walk_begin(g, U.i, a_hi, tile_k, 0, P); walk_valid(w);
+       walk_next(g, w, a_hi, tile_k), ++n) {
     if (n >= max_pairs) return RING_ATTN_EINVAL;
     pairs_out[2 * n] = w.j;
     pairs_out[2 * n + 1] = w.kb;
@@ -379,7 +429,8 @@ int ring_attn_debug_schedule_info(int B, int Hq, int Hkv, int64_t S, int D, int 
     const int64_t a0 = (int64_t)U.tb * BQ;
     const int64_t a_hi = (a0 + BQ - 1 < g.Sq - 1) ? a0 + BQ - 1 : g.Sq - 1;
     int64_t n = 0;
-    for (TileWalk w = walk_begin(g, U.i, a_hi, BN, 0, P); walk_valid(w); walk_next(g, w, a_hi, BN)) {
+    for (TileWalk w = walk_begin(g, U.i, a_hi, BN, 0, P); walk_valid(w);
+         walk_next(g, w, a_hi, BN)) {
       ++n;
       if ((int64_t)w.kb * BN + BN > key_limit(g, U.i, w.j, a0)) ++partial;
     }

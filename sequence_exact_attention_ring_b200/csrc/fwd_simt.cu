@@ -51,8 +51,15 @@ struct Params {
   void* out;
   float* lse;
   float scale;
-  int s_begin, s_end, q_shard_only, partial;
+  int s_begin, s_end, q_shard_only;
+  FwdOut fo;
 };
+
+// Row of local index a of shard i in a [B, H, ., D] input: the whole sequence in token
+// order, or (local) a single shard in shard-local order.
+__device__ __forceinline__ int64_t input_row(const RingGeom& g, bool local, int bh, int i, int64_t a) {
+  return local ? (int64_t)bh * g.Sq + a : (int64_t)bh * g.S + token_of(g, i, a);
+}
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads) ring_fwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k,
@@ -79,7 +86,7 @@ __global__ void __launch_bounds__(kThreads) ring_fwd_simt_kernel(const T* __rest
     const int r = e / D, d = e % D;
     const int64_t aa = a0 + r;
     float val = 0.f;
-    if (aa < g.Sq) val = to_f32<T>(q[((int64_t)bh_q * g.S + token_of(g, U.i, aa)) * D + d]);
+    if (aa < g.Sq) val = to_f32<T>(q[input_row(g, p.fo.local, bh_q, U.i, aa) * D + d]);
     Qs[r * L::kQStride + d] = val;
   }
 
@@ -97,7 +104,7 @@ __global__ void __launch_bounds__(kThreads) ring_fwd_simt_kernel(const T* __rest
       const int64_t b = (int64_t)w.kb * BK + c;
       float kv = 0.f, vv = 0.f;
       if (b < g.Sq) {
-        const int64_t off = ((int64_t)bh_kv * g.S + token_of(g, w.j, b)) * D + d;
+        const int64_t off = input_row(g, p.fo.local, bh_kv, w.j, b) * D + d;
         kv = to_f32<T>(k[off]);
         vv = to_f32<T>(v[off]);
       }
@@ -152,7 +159,38 @@ __global__ void __launch_bounds__(kThreads) ring_fwd_simt_kernel(const T* __rest
   const bool empty = !(l > 0.f);
   const float inv_l = empty ? 0.f : 1.f / l;
   const float lse_v = empty ? -INFINITY : m + logf(l);
-  if (p.partial) {
+  if (p.fo.kind == kOutFold) {
+    // fold this step's row into the running state (weights as in fold_weights of the
+    // tensor-core kernels: lse = ln(e^lse_acc + e^lse_step))
+    const int64_t row = (int64_t)bh_q * g.Sq + a;
+    const float lse_a = p.fo.first ? -INFINITY : p.fo.acc_lse[row];
+    float wa = 0.f, ws = 0.f, lse_n = -INFINITY;
+    if (lse_a != -INFINITY || lse_v != -INFINITY) {
+      const float mx = fmaxf(lse_a, lse_v);
+      const float ea = expf(lse_a - mx), es = expf(lse_v - mx);
+      lse_n = mx + logf(ea + es);
+      wa = ea / (ea + es);
+      ws = es / (ea + es);
+    }
+    if (!(p.fo.first || p.fo.last || lse_v != -INFINITY)) return;  // nothing to add: state unchanged
+    float* acc = p.fo.acc_o + row * D;
+    T* dst = reinterpret_cast<T*>(p.out) + row * D;
+#pragma unroll
+    for (int e = 0; e < NC; ++e) {
+      const float prev = p.fo.first ? 0.f : acc[sub + 4 * e];
+      const float val = wa * prev + ws * (o[e] * inv_l);
+      if (p.fo.last)
+        store_out<T>(dst + sub + 4 * e, val);
+      else
+        acc[sub + 4 * e] = val;
+    }
+    if (sub == 0) {
+      if (p.fo.last)
+        p.lse[row] = lse_n;
+      else
+        p.fo.acc_lse[row] = lse_n;
+    }
+  } else if (p.fo.kind == kOutPartial) {
     float* dst = reinterpret_cast<float*>(p.out) + ((int64_t)bh_q * g.Sq + a) * D;
 #pragma unroll
     for (int e = 0; e < NC; ++e) dst[sub + 4 * e] = o[e] * inv_l;
@@ -182,7 +220,7 @@ static int launch_t(const void* q, const void* k, const void* v, const Params& p
 }  // namespace simt
 
 int launch_fwd_simt(const void* q, const void* k, const void* v, void* out, float* lse, const RingGeom& g,
-                    float scale, int dtype, int s_begin, int s_end, int q_shard_only, int partial,
+                    float scale, int dtype, int s_begin, int s_end, int q_shard_only, const FwdOut& fo,
                     cudaStream_t stream) {
   simt::Params p;
   p.g = g;
@@ -192,7 +230,7 @@ int launch_fwd_simt(const void* q, const void* k, const void* v, void* out, floa
   p.s_begin = s_begin;
   p.s_end = s_end;
   p.q_shard_only = q_shard_only;
-  p.partial = partial;
+  p.fo = fo;
   if (dtype == RING_ATTN_DTYPE_FP32) {
     if (g.D == 64) return simt::launch_t<float, 64>(q, k, v, p, stream);
     if (g.D == 128) return simt::launch_t<float, 128>(q, k, v, p, stream);

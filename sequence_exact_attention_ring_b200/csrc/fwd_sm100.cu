@@ -99,13 +99,13 @@ struct Cfg {
 
 struct Params {
   RingGeom g;
-  void* out;           // final: bf16 [B,Hq,S,D]; partial: fp32 [B,Hq,Sq,D]
-  float* lse;          // final: [B,Hq,S];      partial: [B,Hq,Sq]
+  void* out;           // final: bf16 [B,Hq,S,D]; partial: fp32 [B,Hq,Sq,D]; last fold step: bf16 [B,Hq,Sq,D]
+  float* lse;          // final: [B,Hq,S];      partial, fold: [B,Hq,Sq]
   int* status;         // workspace status word
   float scale_log2;    // scale * log2(e)
   int s_begin, s_end;  // ring steps folded by every unit
   int q_shard_only;    // -1: all query shards
-  int partial;         // 1: write the normalised per-step partial (fp32, local order)
+  FwdOut fo;           // output mode and input layout
   uint64_t watchdog_ns;
 };
 
@@ -185,17 +185,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&bars[kQFull], NQ * C::kTileBytes);
         for (int q = 0; q < NQ; ++q) {
           int c1, c2;
-          shard_map_coords(g, U.i, a0 + q * BM, c1, c2);
+          tile_coords(g, p.fo.local, U.i, a0 + q * BM, c1, c2);
           for (int bx = 0; bx < C::kBoxes; ++bx) {
             uint8_t* dst = smem + C::kOffQ + q * C::kTileBytes + bx * C::kBoxBytes;
             tma_load_4d(dst, &tm_q, &bars[kQFull], bx * BOXW, c1, c2, bh_q);
           }
         }
       }
-      for (TileWalk w = walk_begin(g, U.i, a_hi, BN, p.s_begin, p.s_end); walk_valid(w);
-           walk_next(g, w, a_hi, BN)) {
+      for (TileWalk w = walk_begin(g, U.i, a_hi, BN, p.s_begin, p.s_end);
+           walk_valid(w); walk_next(g, w, a_hi, BN)) {
         int c1, c2;
-        shard_map_coords(g, w.j, w.kb * BN, c1, c2);
+        tile_coords(g, p.fo.local, w.j, w.kb * BN, c1, c2);
         for (int kv = 0; kv < 2 && ok; ++kv, ++n) {
           const int slot = n % C::kSlots;
           const uint32_t ph = (uint32_t)(n / C::kSlots) & 1;
@@ -367,10 +367,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool empty_row = !(l > 0.f);
       const float inv_l = empty_row ? 0.f : 1.f / l;
       const float lse_v = empty_row ? NEG_INF : (m_ref + log2f(l)) * 0.69314718055994530942f;
-      const int64_t tok = token_of(g, U.i, a);
-      const int64_t out_row = p.partial ? (int64_t)bh_q * g.Sq + a : (int64_t)bh_q * g.S + tok;
-      store_row<D>(tO, n > 0, row_ok, inv_l, p.partial, p.out, out_row);
-      if (row_ok) p.lse[out_row] = lse_v;
+      if (p.fo.kind == kOutFold) {
+        fold_row<D>(tO, n > 0, row_ok, inv_l, lse_v, p.fo.first, p.fo.last, p.fo.acc_o, p.fo.acc_lse, p.out, p.lse,
+                    (int64_t)bh_q * g.Sq + a);
+      } else {
+        const bool partial = p.fo.kind == kOutPartial;
+        const int64_t out_row = partial ? (int64_t)bh_q * g.Sq + a : (int64_t)bh_q * g.S + token_of(g, U.i, a);
+        store_row<D>(tO, n > 0, row_ok, inv_l, partial, p.out, out_row);
+        if (row_ok) p.lse[out_row] = lse_v;
+      }
     }
   }
 
@@ -385,14 +390,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ------------------------------------------------------------------------------ host
 template <int D>
 static int launch_impl(const void* q, const void* k, const void* v, void* out, float* lse, const RingGeom& g,
-                       float scale, int s_begin, int s_end, int q_shard_only, int partial, int* status,
+                       float scale, int s_begin, int s_end, int q_shard_only, const FwdOut& fo, int* status,
                        uint64_t watchdog_ns, cudaStream_t stream) {
   using C = Cfg<D>;
   CUtensorMap mq, mk, mv;
   int rc;
-  if ((rc = encode_shard_map(&mq, q, g, g.Hq, D, BM)) != 0) return rc;
-  if ((rc = encode_shard_map(&mk, k, g, g.Hkv, D, BN)) != 0) return rc;
-  if ((rc = encode_shard_map(&mv, v, g, g.Hkv, D, BN)) != 0) return rc;
+  const bool local = fo.local != 0;
+  if ((rc = encode_input_map(&mq, q, g, local, g.Hq, D, BM)) != 0) return rc;
+  if ((rc = encode_input_map(&mk, k, g, local, g.Hkv, D, BN)) != 0) return rc;
+  if ((rc = encode_input_map(&mv, v, g, local, g.Hkv, D, BN)) != 0) return rc;
   Params p;
   p.g = g;
   p.out = out;
@@ -402,7 +408,7 @@ static int launch_impl(const void* q, const void* k, const void* v, void* out, f
   p.s_begin = s_begin;
   p.s_end = s_end;
   p.q_shard_only = q_shard_only;
-  p.partial = partial;
+  p.fo = fo;
   p.watchdog_ns = watchdog_ns;
   if (cudaFuncSetAttribute(ring_fwd_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            C::kSmemBytes) != cudaSuccess)
@@ -422,13 +428,13 @@ static int launch_impl(const void* q, const void* k, const void* v, void* out, f
 }  // namespace sm100
 
 int launch_fwd_sm100(const void* q, const void* k, const void* v, void* out, float* lse, const RingGeom& g,
-                     float scale, int s_begin, int s_end, int q_shard_only, int partial, int* status,
+                     float scale, int s_begin, int s_end, int q_shard_only, const FwdOut& fo, int* status,
                      uint64_t watchdog_ns, cudaStream_t stream) {
   if (g.D == 128)
-    return sm100::launch_impl<128>(q, k, v, out, lse, g, scale, s_begin, s_end, q_shard_only, partial, status,
+    return sm100::launch_impl<128>(q, k, v, out, lse, g, scale, s_begin, s_end, q_shard_only, fo, status,
                                    watchdog_ns, stream);
   if (g.D == 64)
-    return sm100::launch_impl<64>(q, k, v, out, lse, g, scale, s_begin, s_end, q_shard_only, partial, status,
+    return sm100::launch_impl<64>(q, k, v, out, lse, g, scale, s_begin, s_end, q_shard_only, fo, status,
                                   watchdog_ns, stream);
   return RING_ATTN_EUNSUPPORTED;
 }

@@ -82,13 +82,13 @@ constexpr uint32_t kIdescPV = idesc_bf16_f32(2 * BM, D, 0, 1);
 
 struct Params {
   RingGeom g;
-  void* out;
+  void* out;      // see FwdOut: final, per-step partial or (last fold step) shard-local bf16
   float* lse;
   int* status;
   float scale_log2;
   int s_begin, s_end;
   int q_shard_only;
-  int partial;
+  FwdOut fo;
   uint64_t watchdog_ns;
 };
 
@@ -163,14 +163,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (int q = 0; q < NQ && ok; ++q) {
         const int row = (int)(a0 + 256 * q + 128 * rank);
         int c1, c2;
-        shard_map_coords(g, U.i, row, c1, c2);
+        tile_coords(g, p.fo.local, U.i, row, c1, c2);
         for (int bx = 0; bx < 2; ++bx) {
           uint8_t* dst = smem + kOffQ + q * kQTileBytes + bx * kQBoxBytes;
           tma_load_4d_2sm(dst, &tm_q, leader_q, bx * BOXW, c1, c2, bh_q);
         }
       }
-      for (TileWalk w = walk_begin(g, U.i, a_hi, BN, p.s_begin, p.s_end); walk_valid(w) && ok;
-           walk_next(g, w, a_hi, BN)) {
+      for (TileWalk w = walk_begin(g, U.i, a_hi, BN, p.s_begin, p.s_end);
+           walk_valid(w) && ok; walk_next(g, w, a_hi, BN)) {
         for (int kv = 0; kv < 2; ++kv, ++n) {
           const int slot = n % kSlots;
           const uint32_t ph = (uint32_t)(n / kSlots) & 1;
@@ -181,13 +181,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           if (kv == 0) {
             // K half: keys [64 r, 64 r + 64) of the tile, all 128 dims (two 64-dim boxes)
             int c1, c2;
-            shard_map_coords(g, w.j, w.kb * BN + 64 * (int)rank, c1, c2);
+            tile_coords(g, p.fo.local, w.j, w.kb * BN + 64 * (int)rank, c1, c2);
             for (int bx = 0; bx < 2; ++bx)
               tma_load_4d_2sm(dst + bx * kKBoxBytes, &tm_k, leader_full, bx * BOXW, c1, c2, bh_kv);
           } else {
             // V half: all 128 keys of the tile, dims [64 r, 64 r + 64)
             int c1, c2;
-            shard_map_coords(g, w.j, w.kb * BN, c1, c2);
+            tile_coords(g, p.fo.local, w.j, w.kb * BN, c1, c2);
             tma_load_4d_2sm(dst, &tm_v, leader_full, 64 * (int)rank, c1, c2, bh_kv);
           }
         }
@@ -361,10 +361,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const bool empty_row = !(l > 0.f);
       const float inv_l = empty_row ? 0.f : 1.f / l;
       const float lse_v = empty_row ? NEG_INF : (m_ref + log2f(l)) * 0.69314718055994530942f;
-      const int64_t tok = token_of(g, U.i, a);
-      const int64_t out_row = p.partial ? (int64_t)bh_q * g.Sq + a : (int64_t)bh_q * g.S + tok;
-      store_row<D>(tO, n > 0, row_ok, inv_l, p.partial, p.out, out_row);
-      if (row_ok) p.lse[out_row] = lse_v;
+      if (p.fo.kind == kOutFold) {
+        fold_row<D>(tO, n > 0, row_ok, inv_l, lse_v, p.fo.first, p.fo.last, p.fo.acc_o, p.fo.acc_lse, p.out, p.lse,
+                    (int64_t)bh_q * g.Sq + a);
+      } else {
+        const bool partial = p.fo.kind == kOutPartial;
+        const int64_t out_row = partial ? (int64_t)bh_q * g.Sq + a : (int64_t)bh_q * g.S + token_of(g, U.i, a);
+        store_row<D>(tO, n > 0, row_ok, inv_l, partial, p.out, out_row);
+        if (row_ok) p.lse[out_row] = lse_v;
+      }
     }
   }
 
@@ -380,15 +385,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 }  // namespace sm100x2
 
 int launch_fwd_sm100_2sm(const void* q, const void* k, const void* v, void* out, float* lse, const RingGeom& g,
-                         float scale, int s_begin, int s_end, int q_shard_only, int partial, int* status,
+                         float scale, int s_begin, int s_end, int q_shard_only, const FwdOut& fo, int* status,
                          uint64_t watchdog_ns, cudaStream_t stream) {
   using namespace sm100x2;
   if (g.D != D) return RING_ATTN_EUNSUPPORTED;
   CUtensorMap mq, mk, mv;
   int rc;
-  if ((rc = encode_shard_map(&mq, q, g, g.Hq, D, BM)) != 0) return rc;
-  if ((rc = encode_shard_map(&mk, k, g, g.Hkv, D, 64)) != 0) return rc;
-  if ((rc = encode_shard_map(&mv, v, g, g.Hkv, D, BN)) != 0) return rc;
+  const bool local = fo.local != 0;
+  if ((rc = encode_input_map(&mq, q, g, local, g.Hq, D, BM)) != 0) return rc;
+  if ((rc = encode_input_map(&mk, k, g, local, g.Hkv, D, 64)) != 0) return rc;
+  if ((rc = encode_input_map(&mv, v, g, local, g.Hkv, D, BN)) != 0) return rc;
   Params p;
   p.g = g;
   p.out = out;
@@ -398,7 +404,7 @@ int launch_fwd_sm100_2sm(const void* q, const void* k, const void* v, void* out,
   p.s_begin = s_begin;
   p.s_end = s_end;
   p.q_shard_only = q_shard_only;
-  p.partial = partial;
+  p.fo = fo;
   p.watchdog_ns = watchdog_ns;
   if (cudaFuncSetAttribute(ring_fwd_sm100_2sm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
       cudaSuccess)

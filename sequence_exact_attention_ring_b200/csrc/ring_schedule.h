@@ -68,6 +68,19 @@ RA_HD void shard_map_coords(const RingGeom& g, int i, int64_t a, int& c1, int& c
   }
 }
 
+// Tensor-map coordinates of local row a of shard i: in the sharded view of the whole
+// sequence (shard_map_coords), or, when the tensor holds only that one shard in
+// shard-local order (a device of a multi-GPU ring holds one query shard and one KV
+// shard at a time), row a of that buffer.
+RA_HD void tile_coords(const RingGeom& g, bool local, int i, int64_t a, int& c1, int& c2) {
+  if (local) {
+    c1 = (int)a;
+    c2 = 0;
+  } else {
+    shard_map_coords(g, i, a, c1, c2);
+  }
+}
+
 // KV shard met by query shard i at ring step s (0 <= s < P).
 RA_HD int ring_kv_shard(int i, int s, int P) { return (i - s + P) % P; }
 

@@ -16,26 +16,51 @@ typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_
 
 // TMA map of a sharded [B, H, S, D] bf16 tensor (box: 64 elements x box_rows tokens).
 int encode_shard_map(CUtensorMap* map, const void* base, const RingGeom& g, int heads, int D, int box_rows);
+// The same for a single-shard buffer [B, H, Sq, D] in shard-local order when `local`
+// (coordinates from tile_coords), else encode_shard_map.
+int encode_input_map(CUtensorMap* map, const void* base, const RingGeom& g, bool local, int heads, int D,
+                     int box_rows);
 
 // Status word layout at the start of the caller's workspace.
 constexpr size_t kWorkspaceHeaderBytes = 256;
 
-// Fused tcgen05 kernel (bf16). partial=0: final bf16 output in natural token order;
-// partial=1: normalised fp32 per-step partial in shard-local order.
+// How a forward launch reads its inputs and writes its result.
+//   kOutFinal    out in the input dtype [B,Hq,S,D] and lse [B,Hq,S], natural token order
+//   kOutPartial  the normalised per-step partial: fp32 [B,Hq,Sq,D] and lse [B,Hq,Sq],
+//                shard-local order
+//   kOutFold     the step's normalised partial folded into a running state (acc_o fp32
+//                [B,Hq,Sq,D], acc_lse [B,Hq,Sq], shard-local order):
+//                    lse = ln(e^lse_acc + e^lse_step),
+//                    o   = e^(lse_acc - lse) o_acc + e^(lse_step - lse) o_step.
+//                `first`: the state starts from this step (acc is only written);
+//                `last`: the merged rows go to out (input dtype) and lse instead of acc.
+// local: q is one query shard and k, v one KV shard, each a [B, H, Sq, D] buffer in
+// shard-local order (as one device of a multi-GPU ring holds them), instead of the
+// whole sequence in natural token order.
+enum { kOutFinal = 0, kOutPartial = 1, kOutFold = 2 };
+struct FwdOut {
+  int kind;
+  int local;
+  int first, last;
+  float* acc_o;
+  float* acc_lse;
+};
+
+// Fused tcgen05 kernel (bf16), single CTAs, D = 64 or 128.
 int launch_fwd_sm100(const void* q, const void* k, const void* v, void* out, float* lse, const RingGeom& g,
-                     float scale, int s_begin, int s_end, int q_shard_only, int partial, int* status,
+                     float scale, int s_begin, int s_end, int q_shard_only, const FwdOut& fo, int* status,
                      uint64_t watchdog_ns, cudaStream_t stream);
 int64_t fwd_sm100_units(const RingGeom& g, int q_shard_only);
 
 // The same computation on CTA pairs (cta_group::2 MMAs, D = 128 only): each CTA of
 // a pair stages half of every K and V tile.
 int launch_fwd_sm100_2sm(const void* q, const void* k, const void* v, void* out, float* lse, const RingGeom& g,
-                         float scale, int s_begin, int s_end, int q_shard_only, int partial, int* status,
+                         float scale, int s_begin, int s_end, int q_shard_only, const FwdOut& fo, int* status,
                          uint64_t watchdog_ns, cudaStream_t stream);
 
 // fp32-accumulating SIMT kernel (fp32 or bf16 inputs), same schedule and output modes.
 int launch_fwd_simt(const void* q, const void* k, const void* v, void* out, float* lse, const RingGeom& g,
-                    float scale, int dtype, int s_begin, int s_end, int q_shard_only, int partial,
+                    float scale, int dtype, int s_begin, int s_end, int q_shard_only, const FwdOut& fo,
                     cudaStream_t stream);
 
 // Backward pass (bf16, D = 128): the Delta / lse prep kernel, then the dK/dV and dQ

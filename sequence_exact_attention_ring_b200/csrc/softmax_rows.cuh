@@ -195,4 +195,82 @@ __device__ __forceinline__ void store_row(uint32_t tO, bool have_acc, bool row_o
   store_row_cols<D>(tO, have_acc, row_ok, inv_l, partial, out, out_row, D, 0);
 }
 
+// Weights of a running normalised state (lse_a) and of a new normalised partial
+// (lse_s) in their merge: the online-softmax rescale of the RingAttention
+// deep-architecture article (techknowgenie), section 3, applied to states whose l is
+// already divided out. lse = ln(e^lse_a + e^lse_s); an empty side (-inf) gets weight
+// 0; both empty give lse = -inf and weights 0.
+__device__ __forceinline__ void fold_weights(float lse_a, float lse_s, float& wa, float& ws, float& lse) {
+  wa = 0.f;
+  ws = 0.f;
+  lse = -INFINITY;
+  if (lse_a != -INFINITY || lse_s != -INFINITY) {
+    const float mx = fmaxf(lse_a, lse_s);
+    const float ea = expf(lse_a - mx);
+    const float es = expf(lse_s - mx);
+    const float sum = ea + es;
+    lse = mx + logf(sum);
+    wa = ea / sum;
+    ws = es / sum;
+  }
+}
+
+// Folds one row's result of a ring step into the running state (shard-local row
+// `row`): o = wa * acc_o + ws * (O / l), lse = ln(e^lse_acc + e^lse_step). On the
+// first step the state is this step's row; on the last step the merged row goes to
+// `out` (bf16) and `lse_out` instead of the state. A row this step adds nothing to
+// (lse_step = -inf) leaves the state untouched. All lanes execute the tensor-memory
+// loads; only rows that exist are read and written.
+template <int D>
+__device__ __forceinline__ void fold_row(uint32_t tO, bool have_acc, bool row_ok, float inv_l, float lse_step,
+                                         bool first, bool last, float* acc_o, float* acc_lse, void* out,
+                                         float* lse_out, int64_t row) {
+  const float lse_a = (first || !row_ok) ? -INFINITY : acc_lse[row];
+  float wa, ws, lse;
+  fold_weights(lse_a, lse_step, wa, ws, lse);
+  const bool write = row_ok && (first || last || lse_step != -INFINITY);
+  const float wsl = ws * inv_l;
+#pragma unroll 1
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t o[32];
+    if (have_acc) {
+      tmem_ld32(tO + c * 32, o);
+      tmem_wait_ld();
+    }
+    if (!write) continue;
+    const int64_t base = row * D + c * 32;
+    float v[32];
+#pragma unroll
+    for (int e = 0; e < 32; e += 4) {
+      const float4 a4 = first ? make_float4(0.f, 0.f, 0.f, 0.f) : *reinterpret_cast<const float4*>(acc_o + base + e);
+      v[e] = wa * a4.x + (have_acc ? wsl * __uint_as_float(o[e]) : 0.f);
+      v[e + 1] = wa * a4.y + (have_acc ? wsl * __uint_as_float(o[e + 1]) : 0.f);
+      v[e + 2] = wa * a4.z + (have_acc ? wsl * __uint_as_float(o[e + 2]) : 0.f);
+      v[e + 3] = wa * a4.w + (have_acc ? wsl * __uint_as_float(o[e + 3]) : 0.f);
+    }
+    if (last) {
+      uint32_t* dst = reinterpret_cast<uint32_t*>(reinterpret_cast<uint16_t*>(out) + base);
+#pragma unroll
+      for (int e = 0; e < 32; e += 8) {
+        uint4 v4;
+        v4.x = pack_bf16x2(v[e], v[e + 1]);
+        v4.y = pack_bf16x2(v[e + 2], v[e + 3]);
+        v4.z = pack_bf16x2(v[e + 4], v[e + 5]);
+        v4.w = pack_bf16x2(v[e + 6], v[e + 7]);
+        *reinterpret_cast<uint4*>(dst + e / 2) = v4;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; e += 4)
+        *reinterpret_cast<float4*>(acc_o + base + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+    }
+  }
+  if (write) {
+    if (last)
+      lse_out[row] = lse;
+    else
+      acc_lse[row] = lse;
+  }
+}
+
 }  // namespace ringattn

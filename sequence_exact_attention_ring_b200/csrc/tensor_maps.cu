@@ -55,4 +55,15 @@ int encode_shard_map(CUtensorMap* map, const void* base, const RingGeom& g, int 
   return r == CUDA_SUCCESS ? RING_ATTN_OK : RING_ATTN_ECUDA;
 }
 
+int encode_input_map(CUtensorMap* map, const void* base, const RingGeom& g, bool local, int heads, int D,
+                     int box_rows) {
+  if (!local) return encode_shard_map(map, base, g, heads, D, box_rows);
+  // one shard in local order is a contiguous sequence of Sq rows (one shard of P = 1)
+  RingGeom one = g;
+  one.layout = kContiguous;
+  one.S = g.Sq;
+  one.P = 1;
+  return encode_shard_map(map, base, one, heads, D, box_rows);
+}
+
 }  // namespace ringattn

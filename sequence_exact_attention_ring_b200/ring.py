@@ -1,0 +1,278 @@
+"""Exact ring attention spread over ranks: each rank keeps one query shard while the
+KV shards travel around the ring.
+
+RingAttention deep-architecture article (techknowgenie):
+  * section 2 "core principle": with N ranks, rank r keeps query shard r; after each
+    step the KV block it holds moves on to rank (r + 1) mod N and the block of rank
+    (r - 1) mod N arrives, so at step s rank r holds KV shard (r - s) mod N.
+  * section 4 "zero-bubble condition": the next block's transfer hides behind the
+    current block's compute when T_comm <= T_compute (2*2*Sq*D bytes of K and V per
+    head against 4*Sq^2*D FLOPs per block step).
+  * section 5 listing: a current and a next KV buffer, the sends and receives issued
+    on their own stream, a wait before the swap, and the fold of every block into the
+    running (m, l, O) state, with the output produced after the last step.
+  * section "activation checkpointing and memory recomputation": in the backward pass
+    the KV blocks travel the ring the other way, so rank r holds KV shard (r + s) mod N
+    at step s (direction -1 of ring_steps and run_ring_pass).
+
+Every step's attention arithmetic is one ring_attn_fwd_ring_step call: the fused
+kernel, whose epilogue folds the block into the running state. This module only
+orders the transfers and the calls on streams; it moves bytes and never computes
+attention.
+
+Two transports carry the KV shards:
+  * processes, one per GPU, over torch.distributed point-to-point sends and receives
+    (NCCL over NVLink between GPUs; gloo on the host for the bookkeeping tests). The
+    received shard lands in this GPU's own memory and the kernel loads it from there;
+  * virtual ranks inside one process, each with its own buffers and streams on one
+    device: a device-to-device copy on the rank's copy stream pulls the previous rank's
+    current shard into this rank's next buffer while its compute stream runs the step.
+    No kernel of one rank waits on another rank's kernel; streams are ordered by events.
+"""
+from __future__ import annotations
+
+import contextlib
+import math
+
+import torch
+
+from .api import ring_attention_ring_step
+
+_LAYOUTS = ("contiguous", "striped", "zigzag")
+
+
+# ------------------------------------------------------------------ schedule
+
+def ring_steps(rank: int, world: int, direction: int = 1):
+    """The steps of one rank: (step s, KV shard held, rank sent to, rank received from).
+
+    direction +1 is the forward ring (shard (rank - s) mod world at step s, blocks move to
+    rank + 1); -1 the backward ring (shard (rank + s) mod world, blocks move to rank - 1).
+    """
+    if direction not in (1, -1):
+        raise ValueError("direction must be +1 or -1")
+    if not 0 <= rank < world:
+        raise ValueError("rank out of range")
+    return [(s, (rank - direction * s) % world, (rank + direction) % world, (rank - direction) % world)
+            for s in range(world)]
+
+
+# ------------------------------------------------------------------ shard layout helpers
+
+def shard_token_index(S: int, P: int, layout: str, i: int) -> torch.Tensor:
+    """Global tokens of shard i in shard-local order (contiguous: [i*Sq, (i+1)*Sq);
+    striped: a*P + i; zigzag: chunks i and 2P-1-i of C = S/(2P) tokens)."""
+    if layout not in _LAYOUTS or S % P or (layout == "zigzag" and S % (2 * P)):
+        raise ValueError("bad shard geometry")
+    Sq = S // P
+    a = torch.arange(Sq, dtype=torch.int64)
+    if layout == "contiguous":
+        return i * Sq + a
+    if layout == "striped":
+        return a * P + i
+    C = Sq // 2
+    return torch.where(a < C, i * C + a, (2 * P - 1 - i) * C + (a - C))
+
+
+def split_shards(x: torch.Tensor, P: int, layout: str):
+    """[B, H, S, D] in token order -> P contiguous [B, H, Sq, D] shards in shard-local order
+    (input preparation for the ring; each rank of a real ring already holds its shard)."""
+    S = x.shape[2]
+    return [x.index_select(2, shard_token_index(S, P, layout, i).to(x.device)).contiguous() for i in range(P)]
+
+
+def join_shards(shards, layout: str) -> torch.Tensor:
+    """Inverse of split_shards: P shards [B, H, Sq, ...] -> [B, H, S, ...] in token order."""
+    P = len(shards)
+    Sq = shards[0].shape[2]
+    S = P * Sq
+    full = torch.empty((*shards[0].shape[:2], S, *shards[0].shape[3:]), dtype=shards[0].dtype,
+                       device=shards[0].device)
+    for i, sh in enumerate(shards):
+        full.index_copy_(2, shard_token_index(S, P, layout, i).to(sh.device), sh)
+    return full
+
+
+# ------------------------------------------------------------------ one rank per process
+
+def run_ring_pass(k_shard: torch.Tensor, v_shard: torch.Tensor, step_fn, group=None, direction: int = 1,
+                  compute_stream=None, comm_stream=None):
+    """Runs the world_size steps of this rank, passing the (K, V) pair around the ring.
+
+    step_fn(s, kv_index, k_cur, v_cur, first, last) issues step s on the compute stream
+    (the current stream while it runs). Between steps the pair held now is sent to the
+    next rank and the previous rank's pair received into the other buffer, on
+    comm_stream, while step s runs; step s + 1 waits for that transfer. A receive into a
+    buffer waits until the step that read it (two steps earlier) has finished. Every rank
+    takes the same collective steps in the same order. CUDA tensors go through NCCL
+    with streams; CPU tensors (gloo) run the same order synchronously.
+    """
+    import torch.distributed as dist
+
+    rank = dist.get_rank(group)
+    world = dist.get_world_size(group)
+    cuda = k_shard.is_cuda
+    if cuda:
+        compute_stream = compute_stream or torch.cuda.current_stream(k_shard.device)
+        comm_stream = comm_stream or torch.cuda.Stream(k_shard.device)
+        comm_stream.wait_stream(compute_stream)  # the inputs are ready where the caller made them
+    bufs = [(torch.empty_like(k_shard), torch.empty_like(v_shard)) for _ in range(2 if world > 1 else 0)]
+    peer = (lambda r: dist.get_global_rank(group, r)) if group is not None else (lambda r: r)
+    cur = (k_shard, v_shard)
+    compute_done = None
+    for s, j, to, frm in ring_steps(rank, world, direction):
+        works, nxt = [], None
+        if s + 1 < world:
+            nxt = bufs[s % 2]
+            with torch.cuda.stream(comm_stream) if cuda else contextlib.nullcontext():
+                if compute_done is not None:
+                    comm_stream.wait_event(compute_done)  # nxt was read by step s - 1
+                ops = [dist.P2POp(dist.isend, cur[0], peer(to), group), dist.P2POp(dist.isend, cur[1], peer(to), group),
+                       dist.P2POp(dist.irecv, nxt[0], peer(frm), group),
+                       dist.P2POp(dist.irecv, nxt[1], peer(frm), group)]
+                works = dist.batch_isend_irecv(ops)
+        with torch.cuda.stream(compute_stream) if cuda else contextlib.nullcontext():
+            step_fn(s, j, cur[0], cur[1], s == 0, s == world - 1)
+            if cuda:
+                compute_done = torch.cuda.Event()
+                compute_done.record(compute_stream)
+            for w in works:
+                w.wait()  # CUDA: the compute stream waits for the transfer; CPU: blocks
+        if nxt is not None:
+            cur = nxt
+    if cuda:
+        torch.cuda.current_stream(k_shard.device).wait_stream(compute_stream)
+
+
+def ring_attention_distributed(q_shard, k_shard, v_shard, causal: bool = True, layout: str = "striped",
+                               scale: float | None = None, group=None, stream=None, comm_stream=None):
+    """Exact attention with the sequence spread over the ranks of `group`, one shard each.
+
+    Rank r of N holds shard r (under `layout`) of an S = N*Sq token sequence:
+    q_shard [B,Hq,Sq,D] and k_shard/v_shard [B,Hkv,Sq,D], bf16 (or fp32), CUDA, in
+    shard-local order. Returns this rank's (out [B,Hq,Sq,D], lse [B,Hq,Sq]) in
+    shard-local order. The KV shards cross between GPUs by NCCL point-to-point into
+    this GPU's buffers; the kernel reads only this GPU's memory.
+    """
+    import torch.distributed as dist
+
+    rank = dist.get_rank(group)
+    world = dist.get_world_size(group)
+    B, Hq, Sq, D = q_shard.shape
+    S = world * Sq
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    dev = q_shard.device
+    o_acc = torch.empty((B, Hq, Sq, D), dtype=torch.float32, device=dev) if world > 1 else None
+    lse_acc = torch.empty((B, Hq, Sq), dtype=torch.float32, device=dev) if world > 1 else None
+    out = torch.empty_like(q_shard)
+    lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=dev)
+    compute = stream or torch.cuda.current_stream(dev)
+
+    def step(s, j, kc, vc, first, last):
+        ring_attention_ring_step(q_shard, kc, vc, S, world, rank, j, causal, layout, scale, first, last, o_acc,
+                                 lse_acc, out, lse, stream=compute)
+
+    run_ring_pass(k_shard, v_shard, step, group, 1, compute, comm_stream)
+    return out, lse
+
+
+# ------------------------------------------------------------------ virtual ranks on one device
+
+class VirtualRing:
+    """P virtual ranks of the forward ring on one device, each with its own query shard,
+    KV double buffer, running state, workspace, compute stream and copy stream.
+
+    run() issues the P steps of every rank. Rank r's step s folds the KV shard it holds
+    into its state on its compute stream; meanwhile its copy stream pulls the previous
+    rank's current shard into its other buffer (a device-to-device copy). Events order
+    the streams: a copy into a buffer waits for the step and for the neighbour's copy
+    that read it; a step waits for the copy that filled its buffer; a copy waits for the
+    copy that filled its source. No kernel waits on another kernel.
+    """
+
+    def __init__(self, q_shards, k_shards, v_shards, causal=True, layout="striped", scale=None):
+        self.P = len(q_shards)
+        if not (len(k_shards) == len(v_shards) == self.P) or self.P < 1:
+            raise ValueError("one q, k and v shard per rank")
+        B, Hq, Sq, D = q_shards[0].shape
+        self.S = self.P * Sq
+        self.causal, self.layout = causal, layout
+        self.scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+        self.dev = q_shards[0].device
+        self.q, self.k, self.v = list(q_shards), list(k_shards), list(v_shards)
+        P = self.P
+        self.bufs = [[(torch.empty_like(k_shards[r]), torch.empty_like(v_shards[r])) for _ in range(2)]
+                     for r in range(P)] if P > 1 else [[] for _ in range(P)]
+        self.o_acc = [torch.empty((B, Hq, Sq, D), dtype=torch.float32, device=self.dev) for _ in range(P)]
+        self.lse_acc = [torch.empty((B, Hq, Sq), dtype=torch.float32, device=self.dev) for _ in range(P)]
+        self.out = [torch.empty_like(q_shards[r]) for r in range(P)]
+        self.lse = [torch.empty((B, Hq, Sq), dtype=torch.float32, device=self.dev) for _ in range(P)]
+        from . import binding as _b
+        wsb = _b.ring_attn_fwd_workspace_bytes(B, Hq, k_shards[0].shape[1], self.S, D, P, int(causal),
+                                               {"contiguous": 0, "striped": 1, "zigzag": 2}[layout],
+                                               _b.DTYPE_BF16 if q_shards[0].dtype == torch.bfloat16
+                                               else _b.DTYPE_FP32)
+        if wsb == 0:
+            raise _b.RingAttnError(_b.EINVAL, "ring_attn_fwd_workspace_bytes")
+        self.ws = [torch.zeros(wsb, dtype=torch.uint8, device=self.dev) for _ in range(P)]
+        self.compute = [torch.cuda.Stream(self.dev) for _ in range(P)]
+        self.copy = [torch.cuda.Stream(self.dev) for _ in range(P)]
+
+    def _cur(self, r, s):
+        return (self.k[r], self.v[r]) if s == 0 else self.bufs[r][(s - 1) % 2]
+
+    def run(self, timing: bool = False):
+        """Issue every step of every rank; the caller's current stream waits for all of it.
+
+        With timing, returns per-step CUDA events {"compute": [[(start, end)] per step]
+        per rank, "copy": likewise} for the overlap measurement; else None."""
+        P = self.P
+        caller = torch.cuda.current_stream(self.dev)
+        for st in self.compute + self.copy:
+            st.wait_stream(caller)
+        comp_done = [[None] * P for _ in range(P)]
+        copy_done = [[None] * P for _ in range(P)]
+        tm = {"compute": [[] for _ in range(P)], "copy": [[] for _ in range(P)]} if timing else None
+
+        def ev(stream):
+            e = torch.cuda.Event(enable_timing=timing)
+            e.record(stream)
+            return e
+
+        for s in range(P):
+            for r in range(P):
+                cs = self.compute[r]
+                if s > 0:
+                    cs.wait_event(copy_done[r][s - 1])
+                kc, vc = self._cur(r, s)
+                t0 = ev(cs) if timing else None
+                ring_attention_ring_step(self.q[r], kc, vc, self.S, P, r, (r - s) % P, self.causal, self.layout,
+                                         self.scale, s == 0, s == P - 1, self.o_acc[r], self.lse_acc[r], self.out[r],
+                                         self.lse[r], workspace=self.ws[r], stream=cs)
+                comp_done[r][s] = ev(cs)
+                if timing:
+                    tm["compute"][r].append((t0, comp_done[r][s]))
+            if s + 1 < P:
+                for r in range(P):
+                    prev, nxt_rank = (r - 1) % P, (r + 1) % P
+                    xs = self.copy[r]
+                    if s > 0:
+                        xs.wait_event(comp_done[r][s - 1])         # this buffer was read by step s - 1
+                        xs.wait_event(copy_done[prev][s - 1])      # the source was filled at step s - 1
+                        xs.wait_event(copy_done[nxt_rank][s - 1])  # the next rank read this buffer at s - 1
+                    src_k, src_v = self._cur(prev, s)
+                    dst_k, dst_v = self.bufs[r][s % 2]
+                    t0 = ev(xs) if timing else None
+                    with torch.cuda.stream(xs):
+                        dst_k.copy_(src_k, non_blocking=True)
+                        dst_v.copy_(src_v, non_blocking=True)
+                    copy_done[r][s] = ev(xs)
+                    if timing:
+                        tm["copy"][r].append((t0, copy_done[r][s]))
+        for st in self.compute + self.copy:
+            caller.wait_stream(st)
+        return tm
+
+    def results(self):
+        """Per-rank (out [B,Hq,Sq,D], lse [B,Hq,Sq]) in shard-local order."""
+        return list(zip(self.out, self.lse))

@@ -252,3 +252,52 @@ def test_backward_workspace_and_argument_errors(lib):
     bad = list(args)
     bad[13] = 96  # head dim outside {64, 128}
     assert B.ring_attn_bwd(*bad) == B.EUNSUPPORTED
+
+
+def _code_without_comments(path):
+    text = open(path).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return re.sub(r"//[^\n]*", "", text)
+
+
+def test_noalloc_entry_point_calls_no_allocator():
+    """ring_attn_fwd_noalloc and the forward path it calls name no device allocator:
+    the no-allocation file and the forward launch code (C ABI, tensor maps, kernels)."""
+    csrc = os.path.join(ROOT, "sequence_exact_attention_ring_b200", "csrc")
+    files = ["noalloc.cu", "api.cu", "tensor_maps.cu", "fwd_sm100_2sm.cu", "fwd_sm100.cu", "fwd_simt.cu"]
+    banned = re.compile(r"\b(cudaMalloc\w*|cudaFree\w*|cuMemAlloc\w*|cuMemFree\w*|cudaMallocAsync|malloc|new\s)")
+    for f in files:
+        hits = banned.findall(_code_without_comments(os.path.join(csrc, f)))
+        assert not hits, f"{f} names {hits}"
+
+
+def test_noalloc_rejects_bad_arguments_with_the_forward_codes(lib):
+    """Argument errors come back before any CUDA call, with ring_attn_fwd's own code."""
+    vp = ctypes.c_void_p()
+    base = [FAKE] * 5 + [1, 4, 2, 1024, 128, 4, 1, 1, 0.1, 1]
+    for idx, val, code in ((8, 1022, B.EINVAL), (9, 96, B.EUNSUPPORTED), (5, 0, B.EINVAL), (12, 7, B.EINVAL)):
+        a = list(base)
+        a[idx] = val
+        assert lib.ring_attn_fwd_noalloc(*a, None, ctypes.byref(vp)) == code, (idx, val)
+
+
+def test_ring_step_rejects_bad_arguments(lib):
+    """ring_attn_fwd_ring_step argument errors come back before any CUDA call."""
+    ws = FAKE
+
+    def call(o_acc=FAKE, lse_acc=FAKE, out=FAKE, lse_out=FAKE, q=FAKE, i=0, j=1, flags=0, P=4, S=1024, wsb=256,
+             scale=0.1, layout=1):
+        return lib.ring_attn_fwd_ring_step(q, FAKE, FAKE, o_acc, lse_acc, out, lse_out, 1, 4, 2, S, 128, P, i, j, 1,
+                                           layout, ctypes.c_float(scale), 1, flags, ws, wsb, None)
+    assert call(flags=4) == B.EINVAL                      # unknown flag
+    assert call(o_acc=None) == B.EINVAL                   # a middle step needs the state
+    assert call(lse_acc=None, flags=B.STEP_FIRST) == B.EINVAL
+    assert call(out=None, flags=B.STEP_LAST) == B.EINVAL  # a last step needs its outputs
+    assert call(q=None) == B.EINVAL
+    assert call(i=4) == B.EINVAL and call(j=-1) == B.EINVAL
+    assert call(S=1022) == B.EINVAL                       # S % P != 0
+    assert call(o_acc=FAKE + 4) == B.EALIGN
+    assert call(out=FAKE + 2, flags=B.STEP_LAST) == B.EALIGN
+    assert call(wsb=8) == B.EWORKSPACE
+    assert call(scale=-1.0) == B.EINVAL
+    assert call(layout=3) == B.EINVAL

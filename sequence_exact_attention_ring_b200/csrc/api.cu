@@ -331,7 +331,8 @@ int64_t ring_attn_debug_bwd_visit_counts(int64_t S, int P, int causal, int layou
       const Unit U = decode_unit(g, T, -1, uu);
       const int64_t a0 = (int64_t)U.tb * T;
       const int64_t a_hi = (a0 + T - 1 < g.Sq - 1) ? a0 + T - 1 : g.Sq - 1;
-      for (TileWalk w = walk_begin_rev(g, U.i, a_hi, TS); walk_valid(w); walk_next(g, w, a_hi, TS)) {
+      for (TileWalk w = walk_begin_rev(g, U.i, a_hi, TS, launch_anchor(g, -1)); walk_valid(w);
+           walk_next(g, w, a_hi, TS)) {
         ++visits;
         for (int r = 0; r < T && a0 + r < g.Sq; ++r) {
           const int64_t a = a0 + r;
@@ -359,7 +360,7 @@ int64_t ring_attn_debug_visit_counts(int64_t S, int P, int causal, int layout, i
     const Unit U = decode_unit(g, tile_q, -1, u);
     const int64_t a0 = (int64_t)U.tb * tile_q;
     const int64_t a_hi = (a0 + tile_q - 1 < g.Sq - 1) ? a0 + tile_q - 1 : g.Sq - 1;
-    for (TileWalk w = walk_begin(g, U.i, a_hi, tile_k, 0, P); walk_valid(w);
+    for (TileWalk w = walk_begin(g, U.i, a_hi, tile_k, 0, P, launch_anchor(g, -1)); walk_valid(w);
          walk_next(g, w, a_hi, tile_k)) {
       ++tiles;
       for (int64_t a = a0; a < a0 + tile_q && a < g.Sq; ++a) {
@@ -406,7 +407,7 @@ int64_t ring_attn_debug_unit_walk(int B, int Hq, int Hkv, int64_t S, int P, int 
   const int64_t a0 = (int64_t)U.tb * tile_q;
   const int64_t a_hi = (a0 + tile_q - 1 < g.Sq - 1) ? a0 + tile_q - 1 : g.Sq - 1;
   int64_t n = 0;
-  for (TileWalk w = walk_begin(g, U.i, a_hi, tile_k, 0, P); walk_valid(w);
+  for (TileWalk w = walk_begin(g, U.i, a_hi, tile_k, 0, P, launch_anchor(g, -1)); walk_valid(w);
        walk_next(g, w, a_hi, tile_k), ++n) {
     if (n >= max_pairs) return RING_ATTN_EINVAL;
     pairs_out[2 * n] = w.j;
@@ -429,7 +430,7 @@ int ring_attn_debug_schedule_info(int B, int Hq, int Hkv, int64_t S, int D, int 
     const int64_t a0 = (int64_t)U.tb * BQ;
     const int64_t a_hi = (a0 + BQ - 1 < g.Sq - 1) ? a0 + BQ - 1 : g.Sq - 1;
     int64_t n = 0;
-    for (TileWalk w = walk_begin(g, U.i, a_hi, BN, 0, P); walk_valid(w);
+    for (TileWalk w = walk_begin(g, U.i, a_hi, BN, 0, P, launch_anchor(g, -1)); walk_valid(w);
          walk_next(g, w, a_hi, BN)) {
       ++n;
       if ((int64_t)w.kb * BN + BN > key_limit(g, U.i, w.j, a0)) ++partial;

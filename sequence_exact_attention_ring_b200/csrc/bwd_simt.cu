@@ -194,7 +194,7 @@ __global__ void __launch_bounds__(kThreads) dq_kernel(const T* __restrict__ q, c
     dor[e] = row_ok ? ld<T>(dout + off) : 0.f;
     dqr[e] = 0.f;
   }
-  for (TileWalk w = walk_begin_rev(g, U.i, a_hi, TK); walk_valid(w); walk_next(g, w, a_hi, TK)) {
+  for (TileWalk w = walk_begin_rev(g, U.i, a_hi, TK, launch_anchor(g, -1)); walk_valid(w); walk_next(g, w, a_hi, TK)) {
     __syncthreads();
     for (int x = threadIdx.x; x < TK * D; x += kThreads) {
       const int c = x / D, d = x % D;

@@ -478,7 +478,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int c1, c2;
       int64_t m = 0;
       bool ok = true;
-      for (TileWalk w = walk_begin_rev(g, U.i, a_hi, TS); walk_valid(w) && ok; walk_next(g, w, a_hi, TS)) {
+      for (TileWalk w = walk_begin_rev(g, U.i, a_hi, TS, launch_anchor(g, -1)); walk_valid(w) && ok;
+           walk_next(g, w, a_hi, TS)) {
         shard_map_coords(g, w.j, (int64_t)w.kb * TS, c1, c2);
         for (int kind = 0; kind < 2; ++kind, ++m) {
           const int slot = slot_of(m);
@@ -580,7 +581,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     int64_t n = 0;
     bool ok = true;
-    for (TileWalk w = walk_begin_rev(g, U.i, a_hi, TS); walk_valid(w); walk_next(g, w, a_hi, TS), ++n) {
+    for (TileWalk w = walk_begin_rev(g, U.i, a_hi, TS, launch_anchor(g, -1)); walk_valid(w);
+         walk_next(g, w, a_hi, TS), ++n) {
       const int b = (int)(n & 1);
       if (!(ok = mbar_wait(&bars[kB_SFull + b], (uint32_t)((n >> 1) & 1), wd))) break;
       tc_fence_after();

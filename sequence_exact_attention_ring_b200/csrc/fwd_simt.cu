@@ -96,7 +96,7 @@ __global__ void __launch_bounds__(kThreads) ring_fwd_simt_kernel(const T* __rest
   for (int e = 0; e < NC; ++e) o[e] = 0.f;
   float m = -INFINITY, l = 0.f;
 
-  TileWalk w = walk_begin(g, U.i, a_hi, BK, p.s_begin, p.s_end);
+  TileWalk w = walk_begin(g, U.i, a_hi, BK, p.s_begin, p.s_end, launch_anchor(g, p.q_shard_only));
   for (; walk_valid(w); walk_next(g, w, a_hi, BK)) {
     __syncthreads();
     for (int e = tid; e < BK * D; e += kThreads) {

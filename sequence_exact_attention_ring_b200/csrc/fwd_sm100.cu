@@ -192,7 +192,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      for (TileWalk w = walk_begin(g, U.i, a_hi, BN, p.s_begin, p.s_end);
+      for (TileWalk w = walk_begin(g, U.i, a_hi, BN, p.s_begin, p.s_end, launch_anchor(g, p.q_shard_only));
            walk_valid(w); walk_next(g, w, a_hi, BN)) {
         int c1, c2;
         tile_coords(g, p.fo.local, w.j, w.kb * BN, c1, c2);
@@ -303,7 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float l = 0.f;
     int n = 0;
     bool ok = true;
-    TileWalk w = walk_begin(g, U.i, a_hi, BN, p.s_begin, p.s_end);
+    TileWalk w = walk_begin(g, U.i, a_hi, BN, p.s_begin, p.s_end, launch_anchor(g, p.q_shard_only));
     for (; walk_valid(w); walk_next(g, w, a_hi, BN), ++n) {
       if (!(ok = mbar_wait(&bars[kSFull + q], (uint32_t)(n & 1), wd))) break;
       tc_fence_after();

@@ -169,7 +169,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           tma_load_4d_2sm(dst, &tm_q, leader_q, bx * BOXW, c1, c2, bh_q);
         }
       }
-      for (TileWalk w = walk_begin(g, U.i, a_hi, BN, p.s_begin, p.s_end);
+      for (TileWalk w = walk_begin(g, U.i, a_hi, BN, p.s_begin, p.s_end, launch_anchor(g, p.q_shard_only));
            walk_valid(w) && ok; walk_next(g, w, a_hi, BN)) {
         for (int kv = 0; kv < 2; ++kv, ++n) {
           const int slot = n % kSlots;
@@ -297,7 +297,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     float l = 0.f;
     int n = 0;
     bool ok = true;
-    TileWalk w = walk_begin(g, U.i, a_hi, BN, p.s_begin, p.s_end);
+    TileWalk w = walk_begin(g, U.i, a_hi, BN, p.s_begin, p.s_end, launch_anchor(g, p.q_shard_only));
     for (; walk_valid(w); walk_next(g, w, a_hi, BN), ++n) {
       if (!(ok = mbar_wait_cluster(&bars[kSFull + q], (uint32_t)(n & 1), wd))) break;
       tc_fence_after();

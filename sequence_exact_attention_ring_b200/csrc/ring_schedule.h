@@ -124,21 +124,21 @@ RA_HD int kv_tiles_for(const RingGeom& g, int i, int j, int64_t a_hi, int TK) {
 // ring steps [s_begin, s_end). A grid runs its units roughly in index order:
 //   contiguous causal: cost grows with i*nkt + (rows of tb), so units are numbered
 //     longest first by the combined index c = i*nblk + tb, descending;
-//   long sequences (grouped_order: one (b, kv head)'s K and V take >= 32 MiB in
-//     bf16, so the K/V of the heads in flight no longer fits in L2), striped, zigzag
-//     or non-causal: units are grouped by (b, kv head, query shard i); inside a group
-//     the blocks run longest first (tb descending: a block's cost grows with its local
-//     index in these layouts), with the query heads of a GQA group innermost. The
-//     units of a group walk the same ring sequence of KV shards and start together, so
-//     they meet the same K/V tiles at about the same time and L2 serves most of the
-//     re-reads. On the 1M-token causal workloads this halves the DRAM traffic of the
-//     block-major order below; the power it frees raises the clock under the power cap
-//     (striped +4 %, zigzag +6 %);
-//   shorter sequences: longest first over the whole grid, which matters when the grid
-//     is a few waves deep; zigzag causal with whole blocks per chunk walks the 2P
-//     chunks from the last to the first (cost grows with the block's global position);
-//     striped causal and non-causal order by tb descending, inside a tb by (b, kv
-//     head, i, head in the GQA group).
+//   striped causal and every non-causal layout ("block-major"): tb descending (a
+//     block's cost grows with its local index), inside a tb by (b, kv head, i, head in
+//     the GQA group). The units of one (b, kv head, tb) have the same number of key
+//     tiles in every shard (within one tile at the diagonal), so for long sequences
+//     (launch_anchor) they all walk the ring from the same shard and read the same K/V
+//     tiles at about the same time: L2 serves the re-reads of every query shard and
+//     head of the group;
+//   zigzag causal, long sequences (grouped_order: one (b, kv head)'s K and V take
+//     >= 32 MiB in bf16, so the K/V of the heads in flight no longer fits in L2): a
+//     shard's tile counts depend on the query shard here, so units are grouped by
+//     (b, kv head, query shard i), each group's blocks longest first (tb descending),
+//     the query heads of a GQA group innermost; a group walks the same ring sequence
+//     of KV shards and starts together;
+//   zigzag causal, shorter sequences with whole blocks per chunk: the 2P chunks from
+//     the last to the first (cost grows with the block's global position).
 struct Unit {
   int b, h, i, tb;
 };
@@ -179,7 +179,7 @@ RA_HD Unit decode_unit(const RingGeom& g, int BQ, int q_shard_only, int64_t u) {
     r.h = (int)((bg % g.Hkv) * rep + bh % rep);
     return r;
   }
-  if (grouped_order(g)) {
+  if (g.causal && g.layout == kZigzag && grouped_order(g)) {
     int64_t x = u;  // (((b*Hkv + kvh)*P + i)*nblk + (nblk-1-tb))*rep + hr
     const int hr = (int)(x % rep);
     x /= rep;
@@ -225,26 +225,40 @@ RA_HD int64_t unit_tile_count(const RingGeom& g, int i, int64_t a_hi, int TK, in
   return n;
 }
 
+// The shard a full launch's walks count the ring from. In the literal ring, query shard
+// i holds its own KV shard at step 0 (anchor i, the default, -1). On one GPU the fold
+// does not depend on where a query shard's ring starts (exact up to rounding), so for
+// long block-major launches every unit counts the ring from the last shard instead:
+// units of one (b, kv head, tb) then read the same KV shard at the same time. Single
+// ring steps (q_shard_only >= 0) keep the literal step.
+RA_HD int launch_anchor(const RingGeom& g, int q_shard_only) {
+  const bool block_major = g.layout == kStriped || !g.causal;
+  return (q_shard_only < 0 && block_major && grouped_order(g)) ? g.P - 1 : -1;
+}
+
 // Incremental walk over the (ring step, kv tile) sequence of one unit; every role
 // of a kernel advances an identical copy, so they agree on every tile.
 struct TileWalk {
   int s, s_end, j, kb, nkb;
   int i, P;
-  int rev;  // 1: the backward ring, KV shard (i + s) mod P at step s
+  int rev;     // 1: the backward ring, KV shard (anchor + s) mod P at step s
+  int anchor;  // step s holds KV shard (anchor - s) mod P (forward ring)
 };
 
 RA_HD void walk_skip_empty(const RingGeom& g, TileWalk& w, int64_t a_hi, int TK) {
   while (w.s < w.s_end) {
-    w.j = w.rev ? (w.i + w.s) % g.P : ring_kv_shard(w.i, w.s, g.P);
+    w.j = w.rev ? (w.anchor + w.s) % g.P : ring_kv_shard(w.anchor, w.s, g.P);
     w.nkb = kv_tiles_for(g, w.i, w.j, a_hi, TK);
     if (w.nkb > 0) return;
     ++w.s;
   }
 }
 
-RA_HD TileWalk walk_begin(const RingGeom& g, int i, int64_t a_hi, int TK, int s_begin, int s_end) {
+RA_HD TileWalk walk_begin(const RingGeom& g, int i, int64_t a_hi, int TK, int s_begin, int s_end,
+                          int anchor = -1) {
   TileWalk w;
   w.s = s_begin; w.s_end = s_end; w.i = i; w.P = g.P; w.kb = 0; w.j = 0; w.nkb = 0; w.rev = 0;
+  w.anchor = anchor < 0 ? i : anchor;
   walk_skip_empty(g, w, a_hi, TK);
   return w;
 }
@@ -252,10 +266,11 @@ RA_HD TileWalk walk_begin(const RingGeom& g, int i, int64_t a_hi, int TK, int s_
 // The same walk over the backward ring (RingAttention deep-architecture article,
 // techknowgenie, section "activation checkpointing and memory recomputation": KV
 // blocks travel the ring in the opposite direction), so query shard i meets KV
-// shard (i + s) mod P at step s.
-RA_HD TileWalk walk_begin_rev(const RingGeom& g, int i, int64_t a_hi, int TK) {
+// shard (i + s) mod P at step s (counted from `anchor` instead of i when given).
+RA_HD TileWalk walk_begin_rev(const RingGeom& g, int i, int64_t a_hi, int TK, int anchor = -1) {
   TileWalk w;
   w.s = 0; w.s_end = g.P; w.i = i; w.P = g.P; w.kb = 0; w.j = 0; w.nkb = 0; w.rev = 1;
+  w.anchor = anchor < 0 ? i : anchor;
   walk_skip_empty(g, w, a_hi, TK);
   return w;
 }

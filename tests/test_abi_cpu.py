@@ -143,11 +143,16 @@ def test_units_cover_each_block_once_in_launch_order(lib, cfg):
     cost = tab[:, 4]
     # the hook describes the D = 64 geometry: the grouped order starts at S * D >= 2^23
     grouped = S * 64 >= 1 << 23
-    if (causal and layout == 0) or not grouped:
+    if not (causal and layout == 2 and grouped):
+        # contiguous causal, striped causal, non-causal: longest first over the whole grid
         assert (np.diff(cost) <= 0).all(), "units must be launched longest first"
+        if layout == 1 or not causal:
+            # block-major: tb descending, inside a tb by (b, kv head, query shard, head)
+            order = [(-x[3], x[0], x[1] // (Hq // Hkv), x[2], x[1] % (Hq // Hkv)) for x in tab]
+            assert order == sorted(order)
     else:
-        # long sequences, striped or zigzag causal, non-causal: consecutive groups of
-        # nblk * (Hq/Hkv) units share (b, kv head, query shard), blocks longest first
+        # long zigzag causal sequences: consecutive groups of nblk * (Hq/Hkv) units share
+        # (b, kv head, query shard), blocks longest first
         rep = Hq // Hkv
         per = nblk * rep
         groups = set()
@@ -196,6 +201,30 @@ def test_unit_walk_follows_ring_order(lib, layout, causal):
         for j in set(order):
             kbs = pairs[:n][shards == j, 1]
             np.testing.assert_array_equal(kbs, np.arange(len(kbs)))
+
+
+@pytest.mark.parametrize("layout,causal", [(1, 1), (1, 0), (0, 0), (2, 0)])
+def test_long_block_major_walks_share_one_ring_anchor(lib, layout, causal):
+    """Long striped or non-causal launches (S*D >= 2^23): every unit counts the ring from the
+    last shard (step s holds shard (P-1-s) mod P), so units of one block index read the same
+    shard at the same time; the tiles are the same as on the unit's own ring."""
+    S, P = 131072, 8
+    names = {0: "contiguous", 1: "striped", 2: "zigzag"}
+    tab = unit_table(1, 2, 1, S, P, causal, layout)
+    for u in sorted({0, 1, 5, 17, len(tab) // 2, len(tab) - 1}):
+        i, tb = int(tab[u, 2]), int(tab[u, 3])
+        a_hi = min(tb * 256 + 255, S // P - 1)
+        t_hi = int(oracle.shard_tokens(S, P, names[layout], i)[a_hi])
+        expect = []
+        for s_ in range(P):
+            j = (P - 1 - s_) % P
+            toks = oracle.shard_tokens(S, P, names[layout], j)
+            n_keys = int(np.sum(toks <= t_hi)) if causal else S // P
+            expect += [(j, kb) for kb in range((n_keys + 127) // 128)]
+        pairs = np.zeros((len(expect) + 8, 2), dtype=np.int32)
+        n = B.ring_attn_debug_unit_walk(1, 2, 1, S, P, causal, layout, 256, 128, u, pairs.ctypes.data, len(pairs))
+        assert n == len(expect) == tab[u, 4]
+        assert [tuple(x) for x in pairs[:n].tolist()] == expect
 
 
 def test_schedule_info_matches_closed_form_for_1m_striped(lib):

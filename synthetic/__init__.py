@@ -118,6 +118,10 @@ WORKLOADS = {
     "prof_bf16_s256k_striped": Workload("prof_bf16_s256k_striped", "bf16", 1, 8, 8, 262144, 128, 32, True,
                                         "striped", 6, gen_device="cuda",
                                         description="bf16 S=262144 P=32 causal striped (profiling case)"),
+    # the 128k profiling case in the contiguous layout (a shard's rows are adjacent in memory)
+    "prof_bf16_s128k_contig": Workload("prof_bf16_s128k_contig", "bf16", 1, 8, 8, 131072, 128, 32, True,
+                                       "contiguous", 10, gen_device="cuda",
+                                       description="bf16 S=131072 P=32 causal contiguous (profiling case)"),
     "prof_bf16_s512k_striped": Workload("prof_bf16_s512k_striped", "bf16", 1, 8, 8, 524288, 128, 32, True,
                                         "striped", 9, gen_device="cuda",
                                         description="bf16 S=524288 P=32 causal striped (profiling case)"),

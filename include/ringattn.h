@@ -196,6 +196,45 @@ int ring_attn_bwd(const void* q, const void* k, const void* v, const void* out, 
                   void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * The backward pass as one device of a ring spread over devices runs it (RingAttention
+ * deep-architecture article, techknowgenie, section "activation checkpointing and
+ * memory recomputation": each device keeps its query shard, dO and the row statistics;
+ * the K/V shards travel the ring in the reverse direction, each carrying its dK/dV
+ * accumulators, and the attention map is recomputed where they meet). At step s the
+ * device holding query shard i holds KV shard j = (i + s) mod P. The gradients are the
+ * ones ring_attn_bwd computes; every buffer is one shard in shard-local order:
+ *   q_shard, out_shard, dout_shard, dq, dq_acc : [B, Hq,  Sq, D]   (dq_acc fp32, others bf16)
+ *   k_shard, v_shard, dk, dv, dk_acc, dv_acc   : [B, Hkv, Sq, D]   (acc fp32, others bf16)
+ *   lse_shard                                  : [B, Hq,  Sq] fp32, as ring_attn_fwd_ring_step wrote it
+ * ring_attn_bwd_ring_prep computes query shard q_index's row statistics (Delta and lse
+ * in base 2) into `workspace`, once per backward pass; every step of that pass then
+ * uses the same workspace. ring_attn_bwd_ring_step runs the parts asked for:
+ *   RING_ATTN_BWD_PART_KV  KV shard kv_index's dK/dV contributions from query shard
+ *                          q_index, folded into dk_acc/dv_acc (they travel with the shard)
+ *   RING_ATTN_BWD_PART_Q   query shard q_index's dQ contribution from KV shard kv_index,
+ *                          folded into dq_acc
+ * (calling the two parts separately lets the dK/dV accumulators leave for the next
+ * device while the dQ part runs). flags: RING_ATTN_STEP_FIRST starts the accumulators
+ * of the parts run (they are written, not read); RING_ATTN_STEP_LAST writes the summed
+ * gradients in bf16 to dq / dk, dv instead. In a ring both hold at the same steps: the
+ * shard's journey and the device's steps both start at s = 0 and end at s = P - 1.
+ * Supported: bf16, D = 128, an sm_100 device; otherwise RING_ATTN_EUNSUPPORTED.
+ */
+#define RING_ATTN_BWD_PART_KV 1
+#define RING_ATTN_BWD_PART_Q 2
+size_t ring_attn_bwd_ring_workspace_bytes(int B, int Hq, int Hkv, int64_t S, int D, int P,
+                                          int causal, int layout, int dtype);
+int ring_attn_bwd_ring_prep(const void* out_shard, const float* lse_shard, const void* dout_shard,
+                            int B, int Hq, int Hkv, int64_t S, int D, int P, int q_index,
+                            int causal, int layout, int dtype,
+                            void* workspace, size_t workspace_bytes, void* stream);
+int ring_attn_bwd_ring_step(const void* q_shard, const void* dout_shard, const void* k_shard, const void* v_shard,
+                            float* dq_acc, float* dk_acc, float* dv_acc, void* dq, void* dk, void* dv,
+                            int B, int Hq, int Hkv, int64_t S, int D, int P, int q_index, int kv_index,
+                            int causal, int layout, float scale, int dtype, int parts, int flags,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Bytes of device workspace ring_attn_decode needs: the status header plus the
  * split-KV partials (at most 1024 per row). Returns 0 for invalid arguments.
  */

@@ -162,6 +162,62 @@ def ring_attention_backward(q, k, v, out, lse, dout, P: int, causal: bool = True
     return dq, dk, dv
 
 
+def _ptr(t) -> int:
+    return 0 if t is None else t.data_ptr()
+
+
+def ring_backward_prep(out_shard, lse_shard, dout_shard, S: int, P: int, q_index: int, causal: bool = True,
+                       layout="striped", workspace=None, stream=None):
+    """Row statistics of query shard q_index for a backward pass spread over a ring of devices.
+
+    out_shard, dout_shard [B,Hq,Sq,D] bf16 and lse_shard [B,Hq,Sq] fp32 in shard-local order
+    (as ring_attention_ring_step wrote them). Returns the workspace that every
+    ring_backward_step of this pass then uses. Asynchronous on `stream`.
+    """
+    B, Hq, Sq, D = out_shard.shape
+    if Sq * P != S:
+        raise ValueError("shards must hold S / P rows")
+    for t in (out_shard, dout_shard):
+        if not t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous() or t.shape != out_shard.shape:
+            raise ValueError("out_shard and dout_shard must be contiguous bf16 CUDA tensors of one shape")
+    if lse_shard.shape != (B, Hq, Sq) or lse_shard.dtype != torch.float32 or not lse_shard.is_contiguous():
+        raise ValueError("lse_shard must be a contiguous float32 [B, Hq, Sq] tensor")
+    # the key-value head count does not change the statistics' size; use Hq
+    wsb = _b.ring_attn_bwd_ring_workspace_bytes(B, Hq, Hq, S, D, P, int(causal), _layout(layout), _b.DTYPE_BF16)
+    if wsb == 0:
+        raise _b.RingAttnError(_b.EINVAL, "ring_attn_bwd_ring_workspace_bytes")
+    if workspace is None or workspace.numel() < wsb:
+        workspace = torch.empty(wsb, dtype=torch.uint8, device=out_shard.device)
+    rc = _b.ring_attn_bwd_ring_prep(out_shard.data_ptr(), lse_shard.data_ptr(), dout_shard.data_ptr(), B, Hq, Hq, S, D,
+                                    P, q_index, int(causal), _layout(layout), _b.DTYPE_BF16, workspace.data_ptr(),
+                                    workspace.numel(), _stream_ptr(stream))
+    _b.check(rc, "ring_attn_bwd_ring_prep")
+    return workspace
+
+
+def ring_backward_step(q_shard, dout_shard, k_shard, v_shard, S: int, P: int, q_index: int, kv_index: int,
+                       workspace, causal: bool = True, layout="striped", scale: float | None = None, parts=3,
+                       first: bool = False, last: bool = False, dq_acc=None, dk_acc=None, dv_acc=None, dq=None,
+                       dk=None, dv=None, stream=None):
+    """One step of the backward ring: the dK/dV contributions of query shard q_index to KV
+    shard kv_index (parts & 1, folded into dk_acc/dv_acc) and/or the dQ contribution of KV
+    shard kv_index to query shard q_index (parts & 2, folded into dq_acc). Accumulators are
+    fp32, started on `first`; on `last` the bf16 gradients are written to dq / dk, dv.
+    All tensors are single shards in shard-local order. Asynchronous on `stream`."""
+    _check_qkv(q_shard, k_shard, v_shard)
+    B, Hq, Sq, D = q_shard.shape
+    if Sq * P != S:
+        raise ValueError("shards must hold S / P rows")
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    flags = (_b.STEP_FIRST if first else 0) | (_b.STEP_LAST if last else 0)
+    rc = _b.ring_attn_bwd_ring_step(q_shard.data_ptr(), dout_shard.data_ptr(), k_shard.data_ptr(), v_shard.data_ptr(),
+                                    _ptr(dq_acc), _ptr(dk_acc), _ptr(dv_acc), _ptr(dq), _ptr(dk), _ptr(dv), B, Hq,
+                                    k_shard.shape[1], S, D, P, q_index, kv_index, int(causal), _layout(layout), scale,
+                                    _DTYPES[q_shard.dtype], int(parts), flags, workspace.data_ptr(),
+                                    workspace.numel(), _stream_ptr(stream))
+    _b.check(rc, "ring_attn_bwd_ring_step")
+
+
 def ring_attention_decode(q1, k, v, P: int, layout="striped", scale: float | None = None, workspace=None,
                           stream=None):
     """One decode step: q1 [B, Hq, D] (one new row per head) against the cache k, v [B, Hkv, S, D]

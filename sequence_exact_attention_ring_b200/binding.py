@@ -31,6 +31,8 @@ ALGO_TCGEN05 = 2
 ALGO_TCGEN05_1SM = 3
 STEP_FIRST = 1
 STEP_LAST = 2
+BWD_PART_KV = 1
+BWD_PART_Q = 2
 
 _c_int, _c_i64, _c_size, _vp, _c_float = ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_float
 
@@ -55,6 +57,13 @@ SIGNATURES = {
                                                 _c_int]),
     "ring_attn_bwd": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_i64, _c_int,
                                _c_int, _c_int, _c_int, _c_float, _c_int, _vp, _c_size, _vp]),
+    "ring_attn_bwd_ring_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int, _c_i64, _c_int, _c_int, _c_int,
+                                                     _c_int, _c_int]),
+    "ring_attn_bwd_ring_prep": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_i64, _c_int, _c_int, _c_int,
+                                         _c_int, _c_int, _c_int, _vp, _c_size, _vp]),
+    "ring_attn_bwd_ring_step": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int,
+                                         _c_i64, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int,
+                                         _c_int, _c_int, _vp, _c_size, _vp]),
     "ring_attn_decode_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int, _c_i64, _c_int, _c_int, _c_int, _c_int]),
     "ring_attn_decode": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_i64, _c_int, _c_int, _c_int,
                                   _c_float, _c_int, _vp, _c_size, _vp]),
@@ -161,6 +170,24 @@ def ring_attn_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, Hq, Hkv, S, D, P, caus
                   workspace_bytes, stream) -> int:
     return load().ring_attn_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, Hq, Hkv, S, D, P, causal, layout, scale,
                                 dtype, workspace, workspace_bytes, stream)
+
+
+def ring_attn_bwd_ring_workspace_bytes(B, Hq, Hkv, S, D, P, causal, layout, dtype) -> int:
+    return load().ring_attn_bwd_ring_workspace_bytes(B, Hq, Hkv, S, D, P, causal, layout, dtype)
+
+
+def ring_attn_bwd_ring_prep(out_shard, lse_shard, dout_shard, B, Hq, Hkv, S, D, P, q_index, causal, layout, dtype,
+                            workspace, workspace_bytes, stream) -> int:
+    return load().ring_attn_bwd_ring_prep(out_shard, lse_shard, dout_shard, B, Hq, Hkv, S, D, P, q_index, causal,
+                                          layout, dtype, workspace, workspace_bytes, stream)
+
+
+def ring_attn_bwd_ring_step(q_shard, dout_shard, k_shard, v_shard, dq_acc, dk_acc, dv_acc, dq, dk, dv, B, Hq, Hkv, S,
+                            D, P, q_index, kv_index, causal, layout, scale, dtype, parts, flags, workspace,
+                            workspace_bytes, stream) -> int:
+    return load().ring_attn_bwd_ring_step(q_shard, dout_shard, k_shard, v_shard, dq_acc, dk_acc, dv_acc, dq, dk, dv,
+                                          B, Hq, Hkv, S, D, P, q_index, kv_index, causal, layout, scale, dtype, parts,
+                                          flags, workspace, workspace_bytes, stream)
 
 
 def ring_attn_decode_workspace_bytes(B, Hq, Hkv, S, D, P, layout, dtype) -> int:

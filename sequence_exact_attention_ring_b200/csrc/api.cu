@@ -262,6 +262,75 @@ int ring_attn_bwd(const void* q, const void* k, const void* v, const void* out, 
   return launch_bwd_simt(q, k, v, out, lse, dout, dq, dk, dv, g, scale, dtype, stats, st);
 }
 
+size_t ring_attn_bwd_ring_workspace_bytes(int B, int Hq, int Hkv, int64_t S, int D, int P, int causal, int layout,
+                                          int dtype) {
+  RingGeom g;
+  if (check_geom(B, Hq, Hkv, S, D, P, causal, layout, dtype, &g) != RING_ATTN_OK) return 0;
+  return kWorkspaceHeaderBytes + 2 * sizeof(float) * (size_t)bwd_ring_stat_rows(g);
+}
+
+namespace {
+int check_bwd_ring(int B, int Hq, int Hkv, int64_t S, int D, int P, int q_index, int causal, int layout, int dtype,
+                   void* workspace, size_t workspace_bytes, RingGeom* g) {
+  int rc = check_geom(B, Hq, Hkv, S, D, P, causal, layout, dtype, g);
+  if (rc) return rc;
+  if (q_index < 0 || q_index >= P) return RING_ATTN_EINVAL;
+  const size_t need = ring_attn_bwd_ring_workspace_bytes(B, Hq, Hkv, S, D, P, causal, layout, dtype);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return RING_ATTN_EWORKSPACE;
+  if (dtype != RING_ATTN_DTYPE_BF16 || D != 128 || !device_is_sm100()) return RING_ATTN_EUNSUPPORTED;
+  return RING_ATTN_OK;
+}
+}  // namespace
+
+int ring_attn_bwd_ring_prep(const void* out_shard, const float* lse_shard, const void* dout_shard, int B, int Hq,
+                            int Hkv, int64_t S, int D, int P, int q_index, int causal, int layout, int dtype,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  if (!out_shard || !lse_shard || !dout_shard) return RING_ATTN_EINVAL;
+  RingGeom g;
+  int rc = check_bwd_ring(B, Hq, Hkv, S, D, P, q_index, causal, layout, dtype, workspace, workspace_bytes, &g);
+  if (rc) return rc;
+  if (!aligned16(out_shard) || !aligned16(lse_shard) || !aligned16(dout_shard)) return RING_ATTN_EALIGN;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((rc = reset_status(workspace, st))) return rc;
+  float* stats = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kWorkspaceHeaderBytes);
+  return launch_bwd_ring_prep(out_shard, lse_shard, dout_shard, g, q_index, stats, st);
+}
+
+int ring_attn_bwd_ring_step(const void* q_shard, const void* dout_shard, const void* k_shard, const void* v_shard,
+                            float* dq_acc, float* dk_acc, float* dv_acc, void* dq, void* dk, void* dv, int B, int Hq,
+                            int Hkv, int64_t S, int D, int P, int q_index, int kv_index, int causal, int layout,
+                            float scale, int dtype, int parts, int flags, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  RingGeom g;
+  int rc = check_geom(B, Hq, Hkv, S, D, P, causal, layout, dtype, &g);
+  if (rc) return rc;
+  if (kv_index < 0 || kv_index >= P) return RING_ATTN_EINVAL;
+  if (parts < 1 || parts > (RING_ATTN_BWD_PART_KV | RING_ATTN_BWD_PART_Q)) return RING_ATTN_EINVAL;
+  if (flags & ~(RING_ATTN_STEP_FIRST | RING_ATTN_STEP_LAST)) return RING_ATTN_EINVAL;
+  const bool first = (flags & RING_ATTN_STEP_FIRST) != 0;
+  const bool last = (flags & RING_ATTN_STEP_LAST) != 0;
+  const bool need_acc = !(first && last);
+  const bool kv = (parts & RING_ATTN_BWD_PART_KV) != 0;
+  const bool qp = (parts & RING_ATTN_BWD_PART_Q) != 0;
+  if (!q_shard || !dout_shard || !k_shard || !v_shard) return RING_ATTN_EINVAL;
+  if (kv && ((need_acc && (!dk_acc || !dv_acc)) || (last && (!dk || !dv)))) return RING_ATTN_EINVAL;
+  if (qp && ((need_acc && !dq_acc) || (last && !dq))) return RING_ATTN_EINVAL;
+  if (!aligned16(q_shard) || !aligned16(dout_shard) || !aligned16(k_shard) || !aligned16(v_shard))
+    return RING_ATTN_EALIGN;
+  if ((dk_acc && !aligned16(dk_acc)) || (dv_acc && !aligned16(dv_acc)) || (dq_acc && !aligned16(dq_acc)) ||
+      (dq && !aligned16(dq)) || (dk && !aligned16(dk)) || (dv && !aligned16(dv)))
+    return RING_ATTN_EALIGN;
+  if (!(scale > 0.f) || !isfinite(scale)) return RING_ATTN_EINVAL;
+  if ((rc = check_bwd_ring(B, Hq, Hkv, S, D, P, q_index, causal, layout, dtype, workspace, workspace_bytes, &g)))
+    return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((rc = reset_status(workspace, st))) return rc;
+  float* stats = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kWorkspaceHeaderBytes);
+  return launch_bwd_ring_step_sm100(q_shard, dout_shard, k_shard, v_shard, dq_acc, dk_acc, dv_acc, dq, dk, dv, g,
+                                    q_index, kv_index, scale, parts, first, last, stats, static_cast<int*>(workspace),
+                                    watchdog_ns(), st);
+}
+
 size_t ring_attn_decode_workspace_bytes(int B, int Hq, int Hkv, int64_t S, int D, int P, int layout, int dtype) {
   RingGeom g;
   if (check_geom(B, Hq, Hkv, S, D, P, 0, layout, dtype, &g) != RING_ATTN_OK) return 0;

@@ -85,17 +85,19 @@ __device__ __forceinline__ uint64_t mnmajor_step(uint64_t base, int k) {
 // ----------------------------------------------------------------------- prep
 // One warp per padded shard-local query row (bh, i, a): lse2 = lse * log2(e) and
 // delta = <dO_t, O_t> in fp32 for t = token_of(i, a); rows a >= Sq get +inf and 0.
+// local_i >= 0: out, dout and lse hold only query shard local_i, in shard-local order,
+// and the statistics are laid out for that one shard ([B*Hq][1][sq_pad]).
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint16_t* __restrict__ out,
                                                        const uint16_t* __restrict__ dout,
                                                        const float* __restrict__ lse, float* __restrict__ lse2,
                                                        float* __restrict__ delta, RingGeom g, int64_t sq_pad,
-                                                       int64_t rows) {
+                                                       int64_t rows, int local_i) {
   const int64_t row = (int64_t)blockIdx.x * 8 + threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   if (row >= rows) return;
-  const int64_t per_bh = (int64_t)g.P * sq_pad;
+  const int64_t per_bh = (int64_t)(local_i >= 0 ? 1 : g.P) * sq_pad;
   const int64_t bh = row / per_bh;
-  const int i = (int)((row % per_bh) / sq_pad);
+  const int i = local_i >= 0 ? local_i : (int)((row % per_bh) / sq_pad);
   const int64_t a = row % sq_pad;
   if (a >= g.Sq) {
     if (lane == 0) {
@@ -105,7 +107,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint16_t* __restric
     return;
   }
   const int64_t t = token_of(g, i, a);
-  const int64_t base = (bh * g.S + t) * g.D;
+  const int64_t in_row = local_i >= 0 ? bh * g.Sq + a : bh * g.S + t;
+  const int64_t base = in_row * g.D;
   float acc = 0.f;
   for (int d = lane * 4; d < g.D; d += 128) {
     const uint2 o = *reinterpret_cast<const uint2*>(out + base + d);
@@ -118,7 +121,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint16_t* __restric
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
   if (lane == 0) {
-    lse2[row] = lse[bh * g.S + t] * 1.4426950408889634f;
+    lse2[row] = lse[in_row] * 1.4426950408889634f;
     delta[row] = acc;
   }
 }
@@ -136,7 +139,70 @@ struct Params {
   float scale_log2;
   int* status;
   uint64_t watchdog_ns;
+  // One step of a ring spread over devices (step = 1): q, dout, k and v are single-shard
+  // buffers in shard-local order and the statistics cover that one query shard; the dK/dV
+  // pass meets only query shard q_only, the dQ pass units are query shard q_only's and
+  // walk only KV shard kv_only; the epilogues fold into fp32 accumulators acc0 (dK or dQ)
+  // and acc1 (dV), started on `first`, and on `last` write the bf16 results to out0/out1.
+  int step;
+  int q_only, kv_only;
+  int first, last;
+  float* acc0;
+  float* acc1;
 };
+
+// Statistics row of local query row a of shard i, and the memory row of the same query
+// row in q / dout (whole sequence in token order, or one shard in shard-local order).
+__device__ __forceinline__ int64_t stat_row(const Params& p, int bh, int i, int64_t a) {
+  return ((int64_t)bh * (p.step ? 1 : p.g.P) + (p.step ? 0 : i)) * p.sq_pad + a;
+}
+__device__ __forceinline__ int64_t input_row(const Params& p, int bh, int i, int64_t a) {
+  return p.step ? (int64_t)bh * p.g.Sq + a : (int64_t)bh * p.g.S + token_of(p.g, i, a);
+}
+
+// Ring-step epilogue for kCols columns of one row (row stride D): acc = (first ? 0 : acc)
+// + mul * T, with T read from tensor memory; on the last step the sum goes to `out` in
+// bf16 instead. A row this step adds nothing to keeps its accumulator. All lanes execute
+// the tensor-memory loads; only rows that exist are read and written.
+template <int kCols>
+__device__ __forceinline__ void fold_cols(uint32_t tA, bool have, bool row_ok, float mul, bool first, bool last,
+                                          float* acc, void* out, int64_t row, int col0) {
+#pragma unroll 1
+  for (int c = 0; c < kCols / 32; ++c) {
+    uint32_t o[32];
+    if (have) {
+      tmem_ld32(tA + c * 32, o);
+      tmem_wait_ld();
+    }
+    if (!row_ok || (!have && !first && !last)) continue;
+    const int64_t base = row * D + col0 + c * 32;
+    float v[32];
+#pragma unroll
+    for (int e = 0; e < 32; e += 4) {
+      const float4 a4 = first ? make_float4(0.f, 0.f, 0.f, 0.f) : *reinterpret_cast<const float4*>(acc + base + e);
+      v[e] = a4.x + (have ? mul * __uint_as_float(o[e]) : 0.f);
+      v[e + 1] = a4.y + (have ? mul * __uint_as_float(o[e + 1]) : 0.f);
+      v[e + 2] = a4.z + (have ? mul * __uint_as_float(o[e + 2]) : 0.f);
+      v[e + 3] = a4.w + (have ? mul * __uint_as_float(o[e + 3]) : 0.f);
+    }
+    if (last) {
+      uint32_t* dst = reinterpret_cast<uint32_t*>(reinterpret_cast<uint16_t*>(out) + base);
+#pragma unroll
+      for (int e = 0; e < 32; e += 8) {
+        uint4 v4;
+        v4.x = pack_bf16x2(v[e], v[e + 1]);
+        v4.y = pack_bf16x2(v[e + 2], v[e + 3]);
+        v4.z = pack_bf16x2(v[e + 4], v[e + 5]);
+        v4.w = pack_bf16x2(v[e + 6], v[e + 7]);
+        *reinterpret_cast<uint4*>(dst + e / 2) = v4;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; e += 4)
+        *reinterpret_cast<float4*>(acc + base + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+    }
+  }
+}
 
 // P and dS for 32 columns (raw fp32 bits of s and dP), on packed column pairs (f32x2
 // arithmetic): x = s * scale_log2 - lse2,
@@ -247,10 +313,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Watchdog wd{abort_flag, p.status, p.watchdog_ns};
-  const KvUnit U = decode_kv_unit(g, BT, blockIdx.x);
+  const KvUnit U = p.step ? decode_kv_unit_shard(g, BT, blockIdx.x, p.kv_only) : decode_kv_unit(g, BT, blockIdx.x);
   const int bh_kv = U.b * g.Hkv + U.g;
   const int rep = g.Hq / g.Hkv;
-  const int64_t N = qwalk_count(g, U, TS, BT);  // query steps met (x2 loads each)
+  const int q_only = p.step ? p.q_only : -1;
+  const int64_t N = qwalk_count(g, U, TS, BT, q_only);  // query steps met (x2 loads each)
   auto slot_of = [&](int64_t m) { return (int)(m % kA_Slots); };
   auto phase_of = [&](int64_t m) { return (uint32_t)((m / kA_Slots) & 1); };
 
@@ -260,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_do);
       int c1, c2;
-      shard_map_coords(g, U.j, (int64_t)U.kt * BT, c1, c2);
+      tile_coords(g, p.step != 0, U.j, (int64_t)U.kt * BT, c1, c2);
       mbar_arrive_expect_tx(&bars[kA_KVFull], 2 * kTileBytes);
       for (int bx = 0; bx < 2; ++bx) {
         tma_load_4d(smem + kA_OffK + bx * kBoxBytes, &tm_k, &bars[kA_KVFull], bx * BOXW, c1, c2, bh_kv);
@@ -268,11 +335,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       int64_t m = 0;
       bool ok = true;
-      for (QWalk w = qwalk_begin(g, U, TS, BT); qwalk_valid(w) && ok; qwalk_next(g, w, TS)) {
+      for (QWalk w = qwalk_begin(g, U, TS, BT, q_only); qwalk_valid(w) && ok; qwalk_next(g, w, TS)) {
         const int bh_q = U.b * g.Hq + U.g * rep + w.hr;
         const int64_t a0 = (int64_t)w.qt * TS;
-        shard_map_coords(g, w.i, a0, c1, c2);
-        const int64_t stat = ((int64_t)bh_q * g.P + w.i) * p.sq_pad + a0;
+        tile_coords(g, p.step != 0, w.i, a0, c1, c2);
+        const int64_t stat = stat_row(p, bh_q, w.i, a0);
         for (int kind = 0; kind < 2; ++kind, ++m) {
           const int slot = slot_of(m);
           if (!(ok = mbar_wait_backoff<false>(&empty[slot], phase_of(m) ^ 1, wd, kProducerSleepNs))) break;
@@ -357,7 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     int row_i = -1;    // query shard of the cached first visible row
     int64_t row0 = 0;  // first row of shard row_i whose token is >= u
-    for (QWalk w = qwalk_begin(g, U, TS, BT); qwalk_valid(w); qwalk_next(g, w, TS), ++n) {
+    for (QWalk w = qwalk_begin(g, U, TS, BT, q_only); qwalk_valid(w); qwalk_next(g, w, TS), ++n) {
       const int b = (int)(n & 1);
       const int sq = slot_of(2 * n), sd = slot_of(2 * n + 1);
       if (!(ok = mbar_wait(&bars[kA_STFull + b], (uint32_t)((n >> 1) & 1), wd))) break;
@@ -390,10 +457,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (have || n == 0) {
       tc_fence_after();
       const bool row_ok = bk < g.Sq;
-      const int64_t out_row = (int64_t)bh_kv * g.S + (row_ok ? u : 0);
       const uint32_t tAcc = tmem + lane_off + kColAcc + hh * 64;
-      store_row_cols<64>(tAcc, n > 0, row_ok, 1.f, false, p.out1, out_row, D, hh * 64);         // dV
-      store_row_cols<64>(tAcc + D, n > 0, row_ok, p.scale, false, p.out0, out_row, D, hh * 64);  // dK
+      if (p.step) {
+        const int64_t acc_row = (int64_t)bh_kv * g.Sq + bk;  // shard-local
+        fold_cols<64>(tAcc, n > 0, row_ok, 1.f, p.first, p.last, p.acc1, p.out1, acc_row, hh * 64);         // dV
+        fold_cols<64>(tAcc + D, n > 0, row_ok, p.scale, p.first, p.last, p.acc0, p.out0, acc_row, hh * 64);  // dK
+      } else {
+        const int64_t out_row = (int64_t)bh_kv * g.S + (row_ok ? u : 0);
+        store_row_cols<64>(tAcc, n > 0, row_ok, 1.f, false, p.out1, out_row, D, hh * 64);         // dV
+        store_row_cols<64>(tAcc + D, n > 0, row_ok, p.scale, false, p.out0, out_row, D, hh * 64);  // dK
+      }
     }
   }
 
@@ -461,12 +534,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Watchdog wd{abort_flag, p.status, p.watchdog_ns};
-  const Unit U = decode_unit(g, BT, -1, blockIdx.x);
+  const Unit U = decode_unit(g, BT, p.step ? p.q_only : -1, blockIdx.x);
   const int64_t a0 = (int64_t)U.tb * BT;
   const int64_t a_hi = (a0 + BT - 1 < g.Sq - 1) ? a0 + BT - 1 : g.Sq - 1;
   const int bh_q = U.b * g.Hq + U.h;
   const int bh_kv = U.b * g.Hkv + U.h / (g.Hq / g.Hkv);
-  const int64_t N = unit_tile_count(g, U.i, a_hi, TS, 0, g.P);  // the same steps in either ring direction
+  // the backward ring meets KV shard (i + s) mod P at step s: all steps, or in a ring step
+  // the one that meets kv_only (counted from the query shard itself)
+  const int anchor = p.step ? -1 : launch_anchor(g, -1);
+  const int s_lo = p.step ? (p.kv_only - U.i + g.P) % g.P : 0;
+  const int s_hi = p.step ? s_lo + 1 : g.P;
+  const int64_t N = p.step ? kv_tiles_for(g, U.i, p.kv_only, a_hi, TS)
+                           : unit_tile_count(g, U.i, a_hi, TS, 0, g.P);  // the same steps in either ring direction
   auto slot_of = [&](int64_t m) { return (int)(m % kB_Slots); };
   auto phase_of = [&](int64_t m) { return (uint32_t)((m / kB_Slots) & 1); };
 
@@ -478,9 +557,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int c1, c2;
       int64_t m = 0;
       bool ok = true;
-      for (TileWalk w = walk_begin_rev(g, U.i, a_hi, TS, launch_anchor(g, -1)); walk_valid(w) && ok;
+      for (TileWalk w = walk_begin_rev(g, U.i, a_hi, TS, anchor, s_lo, s_hi); walk_valid(w) && ok;
            walk_next(g, w, a_hi, TS)) {
-        shard_map_coords(g, w.j, (int64_t)w.kb * TS, c1, c2);
+        tile_coords(g, p.step != 0, w.j, (int64_t)w.kb * TS, c1, c2);
         for (int kind = 0; kind < 2; ++kind, ++m) {
           const int slot = slot_of(m);
           if (!(ok = mbar_wait_backoff<false>(&empty[slot], phase_of(m) ^ 1, wd, kProducerSleepNs))) break;
@@ -551,7 +630,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int wq = warp % 4, hh = warp / 4;
     const int r = wq * 32 + lane;
     const int64_t a = a0 + r;
-    const int64_t stat = ((int64_t)bh_q * g.P + U.i) * p.sq_pad + a;  // a < sq_pad always
+    const int64_t stat = stat_row(p, bh_q, U.i, a);  // a < sq_pad always
     const float row_lse2 = p.lse2[stat];
     const float row_delta = p.delta[stat];
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
@@ -559,7 +638,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // this thread's row, dims 64 hh .. 64 hh + 63, as 32 bf16 pairs (the memory order);
       // rows past the shard are zeros
       const bool row_ok = a < g.Sq;
-      const int64_t base = ((int64_t)bh_q * g.S + (row_ok ? token_of(g, U.i, a) : 0)) * D + 64 * hh;
+      const int64_t base = (row_ok ? input_row(p, bh_q, U.i, a) : 0) * D + 64 * hh;
       uint32_t x[32];
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
@@ -581,7 +660,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     int64_t n = 0;
     bool ok = true;
-    for (TileWalk w = walk_begin_rev(g, U.i, a_hi, TS, launch_anchor(g, -1)); walk_valid(w);
+    for (TileWalk w = walk_begin_rev(g, U.i, a_hi, TS, anchor, s_lo, s_hi); walk_valid(w);
          walk_next(g, w, a_hi, TS), ++n) {
       const int b = (int)(n & 1);
       if (!(ok = mbar_wait(&bars[kB_SFull + b], (uint32_t)((n >> 1) & 1), wd))) break;
@@ -603,9 +682,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (have || n == 0) {
       tc_fence_after();
       const bool row_ok = a < g.Sq;
-      const int64_t out_row = (int64_t)bh_q * g.S + (row_ok ? token_of(g, U.i, a) : 0);
-      store_row_cols<64>(tmem + lane_off + kColAcc + hh * 64, n > 0, row_ok, p.scale, false, p.out0, out_row, D,
-                         hh * 64);
+      if (p.step) {
+        fold_cols<64>(tmem + lane_off + kColAcc + hh * 64, n > 0, row_ok, p.scale, p.first, p.last, p.acc0, p.out0,
+                      (int64_t)bh_q * g.Sq + a, hh * 64);
+      } else {
+        const int64_t out_row = (int64_t)bh_q * g.S + (row_ok ? token_of(g, U.i, a) : 0);
+        store_row_cols<64>(tmem + lane_off + kColAcc + hh * 64, n > 0, row_ok, p.scale, false, p.out0, out_row, D,
+                           hh * 64);
+      }
     }
   }
 
@@ -621,24 +705,65 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 int64_t bwd_sq_pad(const RingGeom& g) { return (g.Sq + bwd::BT - 1) / bwd::BT * bwd::BT; }
 
+namespace {
+
+bwd::Params base_params(const RingGeom& g, const void* q, const void* dout, float* stats, int64_t stat_rows,
+                        float scale, int* status, uint64_t watchdog_ns) {
+  bwd::Params p;
+  p.g = g;
+  p.q = q;
+  p.dout = dout;
+  p.lse2 = stats;
+  p.delta = stats + stat_rows;
+  p.sq_pad = bwd_sq_pad(g);
+  p.out0 = nullptr;
+  p.out1 = nullptr;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.status = status;
+  p.watchdog_ns = watchdog_ns;
+  p.step = 0;
+  p.q_only = -1;
+  p.kv_only = -1;
+  p.first = 0;
+  p.last = 0;
+  p.acc0 = nullptr;
+  p.acc1 = nullptr;
+  return p;
+}
+
+int set_smem() {
+  using namespace bwd;
+  if (cudaFuncSetAttribute(bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kA_SmemBytes) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kB_SmemBytes) != cudaSuccess)
+    return RING_ATTN_ECUDA;
+  return RING_ATTN_OK;
+}
+
+int launch_prep(const void* out, const float* lse, const void* dout, const RingGeom& g, float* stats, int64_t rows,
+                int local_i, cudaStream_t stream) {
+  const int64_t prep_blocks = (rows + 7) / 8;
+  if (prep_blocks > 0x7fffffff) return RING_ATTN_EINVAL;
+  if (prep_blocks == 0) return RING_ATTN_OK;
+  bwd::bwd_prep_kernel<<<(unsigned)prep_blocks, 256, 0, stream>>>(static_cast<const uint16_t*>(out),
+                                                                    static_cast<const uint16_t*>(dout), lse, stats,
+                                                                    stats + rows, g, bwd_sq_pad(g), rows, local_i);
+  return cudaGetLastError() == cudaSuccess ? RING_ATTN_OK : RING_ATTN_ECUDA;
+}
+
+}  // namespace
+
 int launch_bwd_sm100(const void* q, const void* k, const void* v, const void* out, const float* lse,
                      const void* dout, void* dq, void* dk, void* dv, const RingGeom& g, float scale, float* stats,
                      int* status, uint64_t watchdog_ns, cudaStream_t stream) {
   using namespace bwd;
   if (g.D != D) return RING_ATTN_EUNSUPPORTED;
-  const int64_t sq_pad = bwd_sq_pad(g);
-  const int64_t rows = (int64_t)g.B * g.Hq * g.P * sq_pad;
-  float* lse2 = stats;
-  float* delta = stats + rows;
-  const int64_t prep_blocks = (rows + 7) / 8;
-  if (prep_blocks > 0x7fffffff) return RING_ATTN_EINVAL;
-  bwd_prep_kernel<<<(unsigned)prep_blocks, 256, 0, stream>>>(static_cast<const uint16_t*>(out),
-                                                              static_cast<const uint16_t*>(dout), lse, lse2, delta,
-                                                              g, sq_pad, rows);
-  if (cudaGetLastError() != cudaSuccess) return RING_ATTN_ECUDA;
+  const int64_t rows = (int64_t)g.B * g.Hq * g.P * bwd_sq_pad(g);
+  int rc = launch_prep(out, lse, dout, g, stats, rows, -1, stream);
+  if (rc) return rc;
   // 128-row boxes for the stationary tiles, 64-row boxes for the streamed steps
   CUtensorMap mq, mdo, mk, mv, mq64, mdo64, mk64, mv64;
-  int rc;
   if ((rc = encode_shard_map(&mq, q, g, g.Hq, D, BT)) != 0) return rc;
   if ((rc = encode_shard_map(&mdo, dout, g, g.Hq, D, BT)) != 0) return rc;
   if ((rc = encode_shard_map(&mk, k, g, g.Hkv, D, BT)) != 0) return rc;
@@ -647,21 +772,8 @@ int launch_bwd_sm100(const void* q, const void* k, const void* v, const void* ou
   if ((rc = encode_shard_map(&mdo64, dout, g, g.Hq, D, TS)) != 0) return rc;
   if ((rc = encode_shard_map(&mk64, k, g, g.Hkv, D, TS)) != 0) return rc;
   if ((rc = encode_shard_map(&mv64, v, g, g.Hkv, D, TS)) != 0) return rc;
-  Params p;
-  p.g = g;
-  p.q = q;
-  p.dout = dout;
-  p.lse2 = lse2;
-  p.delta = delta;
-  p.sq_pad = sq_pad;
-  p.scale = scale;
-  p.scale_log2 = scale * 1.4426950408889634f;
-  p.status = status;
-  p.watchdog_ns = watchdog_ns;
-  if (cudaFuncSetAttribute(bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kA_SmemBytes) !=
-          cudaSuccess ||
-      cudaFuncSetAttribute(bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kB_SmemBytes) != cudaSuccess)
-    return RING_ATTN_ECUDA;
+  Params p = base_params(g, q, dout, stats, rows, scale, status, watchdog_ns);
+  if ((rc = set_smem())) return rc;
   const int64_t kv_units = num_kv_units(g, BT);
   const int64_t q_units = num_units(g, BT, -1);
   if (kv_units > 0x7fffffff || q_units > 0x7fffffff) return RING_ATTN_EINVAL;
@@ -673,6 +785,62 @@ int launch_bwd_sm100(const void* q, const void* k, const void* v, const void* ou
   p.out1 = nullptr;
   bwd_dq_kernel<<<(unsigned)q_units, kThreads, kB_SmemBytes, stream>>>(mq, mdo, mk64, mv64, p);
   return cudaGetLastError() == cudaSuccess ? RING_ATTN_OK : RING_ATTN_ECUDA;
+}
+
+int64_t bwd_ring_stat_rows(const RingGeom& g) { return (int64_t)g.B * g.Hq * bwd_sq_pad(g); }
+
+int launch_bwd_ring_prep(const void* out, const float* lse, const void* dout, const RingGeom& g, int q_index,
+                         float* stats, cudaStream_t stream) {
+  if (g.D != bwd::D) return RING_ATTN_EUNSUPPORTED;
+  return launch_prep(out, lse, dout, g, stats, bwd_ring_stat_rows(g), q_index, stream);
+}
+
+int launch_bwd_ring_step_sm100(const void* q, const void* dout, const void* k, const void* v, float* dq_acc,
+                               float* dk_acc, float* dv_acc, void* dq, void* dk, void* dv, const RingGeom& g,
+                               int q_index, int kv_index, float scale, int parts, int first, int last, float* stats,
+                               int* status, uint64_t watchdog_ns, cudaStream_t stream) {
+  using namespace bwd;
+  if (g.D != D) return RING_ATTN_EUNSUPPORTED;
+  const int64_t rows = bwd_ring_stat_rows(g);
+  // single-shard buffers in shard-local order: a 4-D view of one shard of P = 1
+  CUtensorMap mq, mdo, mk, mv, mq64, mdo64, mk64, mv64;
+  int rc;
+  if ((rc = encode_input_map(&mq, q, g, true, g.Hq, D, BT)) != 0) return rc;
+  if ((rc = encode_input_map(&mdo, dout, g, true, g.Hq, D, BT)) != 0) return rc;
+  if ((rc = encode_input_map(&mk, k, g, true, g.Hkv, D, BT)) != 0) return rc;
+  if ((rc = encode_input_map(&mv, v, g, true, g.Hkv, D, BT)) != 0) return rc;
+  if ((rc = encode_input_map(&mq64, q, g, true, g.Hq, D, TS)) != 0) return rc;
+  if ((rc = encode_input_map(&mdo64, dout, g, true, g.Hq, D, TS)) != 0) return rc;
+  if ((rc = encode_input_map(&mk64, k, g, true, g.Hkv, D, TS)) != 0) return rc;
+  if ((rc = encode_input_map(&mv64, v, g, true, g.Hkv, D, TS)) != 0) return rc;
+  Params p = base_params(g, q, dout, stats, rows, scale, status, watchdog_ns);
+  p.step = 1;
+  p.q_only = q_index;
+  p.kv_only = kv_index;
+  p.first = first;
+  p.last = last;
+  if ((rc = set_smem())) return rc;
+  if (parts & RING_ATTN_BWD_PART_KV) {
+    const int64_t kv_units = num_kv_units_shard(g, BT);
+    if (kv_units > 0x7fffffff) return RING_ATTN_EINVAL;
+    p.out0 = dk;
+    p.out1 = dv;
+    p.acc0 = dk_acc;
+    p.acc1 = dv_acc;
+    bwd_dkdv_kernel<<<(unsigned)kv_units, kThreads, kA_SmemBytes, stream>>>(mq64, mdo64, mk, mv, p);
+    if (cudaGetLastError() != cudaSuccess) return RING_ATTN_ECUDA;
+  }
+  if (parts & RING_ATTN_BWD_PART_Q) {
+    const int64_t q_units = num_units(g, BT, q_index);
+    if (q_units > 0x7fffffff) return RING_ATTN_EINVAL;
+    p.out0 = dq;
+    p.out1 = nullptr;
+    p.acc0 = dq_acc;
+    p.acc1 = nullptr;
+    bwd_dq_kernel<<<(unsigned)q_units, kThreads, kB_SmemBytes, stream>>>(mq, mdo, mk64, mv64, p);
+    if (cudaGetLastError() != cudaSuccess) return RING_ATTN_ECUDA;
+  }
+  return RING_ATTN_OK;
 }
 
 }  // namespace ringattn

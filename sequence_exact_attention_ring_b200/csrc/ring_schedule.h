@@ -267,9 +267,10 @@ RA_HD TileWalk walk_begin(const RingGeom& g, int i, int64_t a_hi, int TK, int s_
 // techknowgenie, section "activation checkpointing and memory recomputation": KV
 // blocks travel the ring in the opposite direction), so query shard i meets KV
 // shard (i + s) mod P at step s (counted from `anchor` instead of i when given).
-RA_HD TileWalk walk_begin_rev(const RingGeom& g, int i, int64_t a_hi, int TK, int anchor = -1) {
+RA_HD TileWalk walk_begin_rev(const RingGeom& g, int i, int64_t a_hi, int TK, int anchor = -1, int s_begin = 0,
+                              int s_end = -1) {
   TileWalk w;
-  w.s = 0; w.s_end = g.P; w.i = i; w.P = g.P; w.kb = 0; w.j = 0; w.nkb = 0; w.rev = 1;
+  w.s = s_begin; w.s_end = s_end < 0 ? g.P : s_end; w.i = i; w.P = g.P; w.kb = 0; w.j = 0; w.nkb = 0; w.rev = 1;
   w.anchor = anchor < 0 ? i : anchor;
   walk_skip_empty(g, w, a_hi, TK);
   return w;
@@ -343,6 +344,22 @@ RA_HD KvUnit decode_kv_unit(const RingGeom& g, int TK, int64_t u) {
   return r;
 }
 
+// The KV units of one shard j only (one step of a ring spread over devices: the device
+// holds one KV shard): (b, kv head) innermost, tiles in index order (longest first
+// under a causal mask).
+RA_HD int64_t num_kv_units_shard(const RingGeom& g, int TK) { return (int64_t)g.B * g.Hkv * num_kv_tiles(g, TK); }
+
+RA_HD KvUnit decode_kv_unit_shard(const RingGeom& g, int TK, int64_t u, int j) {
+  const int64_t bg_n = (int64_t)g.B * g.Hkv;
+  KvUnit r;
+  r.kt = (int)(u / bg_n);
+  const int64_t bg = u % bg_n;
+  r.b = (int)(bg / g.Hkv);
+  r.g = (int)(bg % g.Hkv);
+  r.j = j;
+  return r;
+}
+
 // Walk over (query head of the group, ring step, query tile) for one KV tile.
 struct QWalk {
   int hr, rep;  // query head hr of the GQA group
@@ -350,12 +367,13 @@ struct QWalk {
   int qt, nqt;  // current query tile and the shard's tile count
   int qt0;      // first query tile of shard i that sees the KV tile
   int j;
-  int64_t u_min;  // smallest key token of the tile
+  int64_t u_min;   // smallest key token of the tile
+  int s_lo, s_hi;  // the ring steps walked: [0, P), or the one step that meets a single query shard
 };
 
 RA_HD void qwalk_skip_empty(const RingGeom& g, QWalk& w, int TQ) {
   while (w.hr < w.rep) {
-    while (w.s < g.P) {
+    while (w.s < w.s_hi) {
       w.i = (w.j - w.s + g.P) % g.P;
       const int64_t a0 = g.causal ? first_row_at_or_after(g, w.i, w.u_min) : 0;
       if (a0 < g.Sq) {
@@ -365,14 +383,18 @@ RA_HD void qwalk_skip_empty(const RingGeom& g, QWalk& w, int TQ) {
       }
       ++w.s;
     }
-    w.s = 0;
+    w.s = w.s_lo;
     ++w.hr;
   }
 }
 
-RA_HD QWalk qwalk_begin(const RingGeom& g, const KvUnit& U, int TQ, int TK) {
+// q_only >= 0 restricts the walk to the one ring step at which the KV tile meets query
+// shard q_only (one step of a ring spread over devices).
+RA_HD QWalk qwalk_begin(const RingGeom& g, const KvUnit& U, int TQ, int TK, int q_only = -1) {
   QWalk w;
-  w.hr = 0; w.rep = g.Hq / g.Hkv; w.s = 0; w.i = U.j; w.j = U.j;
+  w.s_lo = q_only < 0 ? 0 : (U.j - q_only + g.P) % g.P;
+  w.s_hi = q_only < 0 ? g.P : w.s_lo + 1;
+  w.hr = 0; w.rep = g.Hq / g.Hkv; w.s = w.s_lo; w.i = U.j; w.j = U.j;
   w.nqt = (int)((g.Sq + TQ - 1) / TQ);
   w.qt = 0; w.qt0 = 0;
   w.u_min = token_of(g, U.j, (int64_t)U.kt * TK);
@@ -399,11 +421,12 @@ RA_HD int bwd_first_visible_col(const RingGeom& g, int i, int64_t a0, int64_t u,
 
 // Query tiles one KV unit meets: per shard, the tiles from the first that sees the
 // KV tile's smallest token to the end, for every query head of the group.
-RA_HD int64_t qwalk_count(const RingGeom& g, const KvUnit& U, int TQ, int TK) {
+RA_HD int64_t qwalk_count(const RingGeom& g, const KvUnit& U, int TQ, int TK, int q_only = -1) {
   const int64_t nqt = (g.Sq + TQ - 1) / TQ;
   const int64_t u_min = token_of(g, U.j, (int64_t)U.kt * TK);
   int64_t n = 0;
   for (int i = 0; i < g.P; ++i) {
+    if (q_only >= 0 && i != q_only) continue;
     const int64_t a0 = g.causal ? first_row_at_or_after(g, i, u_min) : 0;
     if (a0 < g.Sq) n += nqt - a0 / TQ;
   }

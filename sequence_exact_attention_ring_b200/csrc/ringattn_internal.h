@@ -70,6 +70,20 @@ int launch_bwd_sm100(const void* q, const void* k, const void* v, const void* ou
                      const void* dout, void* dq, void* dk, void* dv, const RingGeom& g, float scale, float* stats,
                      int* status, uint64_t watchdog_ns, cudaStream_t stream);
 
+// One step of the backward ring spread over devices (bf16, D = 128), on shard-local
+// buffers: the statistics of query shard q_index (launch_bwd_ring_prep, into `stats`:
+// 2 * bwd_ring_stat_rows(g) floats), then per step the dK/dV part (KV shard kv_index's
+// gradients from query shard q_index, folded into dk_acc/dv_acc) and/or the dQ part
+// (query shard q_index's gradient from KV shard kv_index, folded into dq_acc); on the
+// last step the bf16 results go to dq/dk/dv.
+int64_t bwd_ring_stat_rows(const RingGeom& g);
+int launch_bwd_ring_prep(const void* out, const float* lse, const void* dout, const RingGeom& g, int q_index,
+                         float* stats, cudaStream_t stream);
+int launch_bwd_ring_step_sm100(const void* q, const void* dout, const void* k, const void* v, float* dq_acc,
+                               float* dk_acc, float* dv_acc, void* dq, void* dk, void* dv, const RingGeom& g,
+                               int q_index, int kv_index, float scale, int parts, int first, int last, float* stats,
+                               int* status, uint64_t watchdog_ns, cudaStream_t stream);
+
 // Decode (one query row per head against the whole sharded cache, bf16, D = 128):
 // split-KV partials into o_parts [decode_parts(g)][B*Hq][D] and lse_parts, then the
 // merge kernel writes out [B*Hq][D] bf16 and lse [B*Hq].

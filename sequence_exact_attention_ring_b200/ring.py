@@ -176,6 +176,125 @@ def ring_attention_distributed(q_shard, k_shard, v_shard, causal: bool = True, l
     return out, lse
 
 
+def run_backward_ring(k_shard, v_shard, acc_like, step_kv, step_q, group=None, compute_stream=None, comm_stream=None):
+    """The transfers of the backward ring for one rank; returns (dK, dV) of the rank's own
+    KV shard, in K's dtype.
+
+    At step s the rank holds KV shard j = (rank + s) mod world with its dK/dV accumulators
+    (fp32, shaped like `acc_like`). step_kv(s, j, k, v, acc_k, acc_v, fin_k, fin_v, first,
+    last) folds the rank's query shard into them (on the last step into fin_k/fin_v, bf16);
+    step_q(s, j, k, v, first, last) folds KV shard j into the rank's dQ. K and V move on
+    to rank - 1 while step s runs; the accumulators leave once step_kv has run, while
+    step_q runs; the next step waits for both. After the last step each rank holds the
+    finished dK/dV of shard rank - 1 and sends them home. CUDA tensors use NCCL and
+    streams; CPU tensors (gloo) take the same order synchronously.
+    """
+    import torch.distributed as dist
+
+    rank = dist.get_rank(group)
+    world = dist.get_world_size(group)
+    cuda = k_shard.is_cuda
+    if cuda:
+        compute_stream = compute_stream or torch.cuda.current_stream(k_shard.device)
+        comm_stream = comm_stream or torch.cuda.Stream(k_shard.device)
+        comm_stream.wait_stream(compute_stream)
+    peer = (lambda r: dist.get_global_rank(group, r)) if group is not None else (lambda r: r)
+    to, frm = peer((rank - 1) % world), peer((rank + 1) % world)  # blocks move to rank - 1
+    kv_bufs = [(torch.empty_like(k_shard), torch.empty_like(v_shard)) for _ in range(2 if world > 1 else 0)]
+    acc_bufs = [(torch.empty_like(acc_like), torch.empty_like(acc_like)) for _ in range(2 if world > 1 else 0)]
+    fin_k, fin_v = torch.empty_like(k_shard), torch.empty_like(v_shard)
+    cur_kv = (k_shard, v_shard)
+    cur_acc = acc_bufs[0] if world > 1 else (None, None)
+    on_comm = (lambda: torch.cuda.stream(comm_stream)) if cuda else contextlib.nullcontext
+    on_compute = (lambda: torch.cuda.stream(compute_stream)) if cuda else contextlib.nullcontext
+    compute_done = None
+    for s in range(world):
+        j = (rank + s) % world
+        first, last = s == 0, s == world - 1
+        works, nxt_kv, nxt_acc = [], None, None
+        if not last:
+            nxt_kv = kv_bufs[s % 2]
+            with on_comm():
+                if compute_done is not None:
+                    comm_stream.wait_event(compute_done)  # nxt_kv was read by step s - 1
+                works += dist.batch_isend_irecv([
+                    dist.P2POp(dist.isend, cur_kv[0], to, group), dist.P2POp(dist.isend, cur_kv[1], to, group),
+                    dist.P2POp(dist.irecv, nxt_kv[0], frm, group), dist.P2POp(dist.irecv, nxt_kv[1], frm, group)])
+        with on_compute():
+            step_kv(s, j, cur_kv[0], cur_kv[1], cur_acc[0], cur_acc[1], fin_k, fin_v, first, last)
+            if cuda:
+                kv_done = torch.cuda.Event()
+                kv_done.record(compute_stream)
+        if not last:
+            nxt_acc = acc_bufs[(s + 1) % 2]
+            with on_comm():
+                if cuda:
+                    comm_stream.wait_event(kv_done)  # the accumulators leave once this step's part is in
+                works += dist.batch_isend_irecv([
+                    dist.P2POp(dist.isend, cur_acc[0], to, group), dist.P2POp(dist.isend, cur_acc[1], to, group),
+                    dist.P2POp(dist.irecv, nxt_acc[0], frm, group), dist.P2POp(dist.irecv, nxt_acc[1], frm, group)])
+        with on_compute():
+            step_q(s, j, cur_kv[0], cur_kv[1], first, last)
+            if cuda:
+                compute_done = torch.cuda.Event()
+                compute_done.record(compute_stream)
+            for w in works:
+                w.wait()
+        if not last:
+            cur_kv, cur_acc = nxt_kv, nxt_acc
+    if world == 1:
+        return fin_k, fin_v
+    # the shard finished here is rank - 1's: send it home, receive this rank's own
+    home_k, home_v = torch.empty_like(k_shard), torch.empty_like(v_shard)
+    with on_comm():
+        if cuda:
+            comm_stream.wait_stream(compute_stream)
+        works = dist.batch_isend_irecv([
+            dist.P2POp(dist.isend, fin_k, to, group), dist.P2POp(dist.isend, fin_v, to, group),
+            dist.P2POp(dist.irecv, home_k, frm, group), dist.P2POp(dist.irecv, home_v, frm, group)])
+    with on_compute():
+        for w in works:
+            w.wait()
+    if cuda:
+        torch.cuda.current_stream(k_shard.device).wait_stream(compute_stream)
+    return home_k, home_v
+
+
+def ring_attention_backward_distributed(q_shard, k_shard, v_shard, out_shard, lse_shard, dout_shard,
+                                        causal: bool = True, layout: str = "striped", scale: float | None = None,
+                                        group=None, stream=None, comm_stream=None):
+    """Gradients (dq, dk, dv) of this rank's shards for attention spread over the ranks of
+    `group` (the forward of ring_attention_distributed): the backward ring of the
+    RingAttention deep-architecture article, section "activation checkpointing and memory
+    recomputation". All tensors are this rank's shard in shard-local order; out_shard and
+    lse_shard are the forward's results. The per-step arithmetic runs in the library's
+    kernels (ring_attn_bwd_ring_step); this function moves the shards."""
+    import torch.distributed as dist
+
+    from .api import ring_backward_prep, ring_backward_step
+
+    rank = dist.get_rank(group)
+    world = dist.get_world_size(group)
+    B, Hq, Sq, D = q_shard.shape
+    S = world * Sq
+    compute = stream or torch.cuda.current_stream(q_shard.device)
+    ws = ring_backward_prep(out_shard, lse_shard, dout_shard, S, world, rank, causal, layout, stream=compute)
+    dq_acc = torch.empty((B, Hq, Sq, D), dtype=torch.float32, device=q_shard.device) if world > 1 else None
+    dq = torch.empty_like(q_shard)
+    acc_like = torch.empty(k_shard.shape, dtype=torch.float32, device=q_shard.device)
+
+    def step_kv(s, j, kc, vc, acc_k, acc_v, fin_k, fin_v, first, last):
+        ring_backward_step(q_shard, dout_shard, kc, vc, S, world, rank, j, ws, causal, layout, scale, parts=1,
+                           first=first, last=last, dk_acc=acc_k, dv_acc=acc_v, dk=fin_k, dv=fin_v, stream=compute)
+
+    def step_q(s, j, kc, vc, first, last):
+        ring_backward_step(q_shard, dout_shard, kc, vc, S, world, rank, j, ws, causal, layout, scale, parts=2,
+                           first=first, last=last, dq_acc=dq_acc, dq=dq, stream=compute)
+
+    dk, dv = run_backward_ring(k_shard, v_shard, acc_like, step_kv, step_q, group, compute, comm_stream)
+    return dq, dk, dv
+
+
 # ------------------------------------------------------------------ virtual ranks on one device
 
 class VirtualRing:

@@ -330,3 +330,27 @@ def test_ring_step_rejects_bad_arguments(lib):
     assert call(wsb=8) == B.EWORKSPACE
     assert call(scale=-1.0) == B.EINVAL
     assert call(layout=3) == B.EINVAL
+
+
+def test_backward_ring_entry_points_reject_bad_arguments(lib):
+    """ring_attn_bwd_ring_prep / _step argument errors come back before any CUDA call."""
+    wsb = lib.ring_attn_bwd_ring_workspace_bytes(1, 4, 2, 1024, 128, 4, 1, 1, 1)
+    assert wsb == 256 + 2 * 4 * 4 * 256  # header + two statistics of B*Hq*ceil(Sq/128)*128 rows
+    assert lib.ring_attn_bwd_ring_workspace_bytes(1, 4, 2, 1022, 128, 4, 1, 1, 1) == 0
+
+    def step(parts=3, flags=0, i=0, j=1, acc=FAKE, out=FAKE, q=FAKE, ws=FAKE, n=wsb, scale=0.1):
+        return lib.ring_attn_bwd_ring_step(q, FAKE, FAKE, FAKE, acc, acc, acc, out, out, out, 1, 4, 2, 1024, 128, 4,
+                                           i, j, 1, 1, ctypes.c_float(scale), 1, parts, flags, ws, n, None)
+    assert step(parts=0) == B.EINVAL and step(parts=4) == B.EINVAL
+    assert step(flags=4) == B.EINVAL
+    assert step(acc=None) == B.EINVAL                      # a middle step needs the accumulators
+    assert step(out=None, flags=B.STEP_LAST) == B.EINVAL   # a last step needs the outputs
+    assert step(q=None) == B.EINVAL
+    assert step(i=4) == B.EINVAL and step(j=-1) == B.EINVAL
+    assert step(acc=FAKE + 8) == B.EALIGN
+    assert step(n=wsb - 16) == B.EWORKSPACE
+    assert step(scale=0.0) == B.EINVAL
+    prep = lib.ring_attn_bwd_ring_prep
+    assert prep(FAKE, FAKE, FAKE, 1, 4, 2, 1024, 128, 4, 4, 1, 1, 1, FAKE, wsb, None) == B.EINVAL  # q_index
+    assert prep(None, FAKE, FAKE, 1, 4, 2, 1024, 128, 4, 0, 1, 1, 1, FAKE, wsb, None) == B.EINVAL
+    assert prep(FAKE, FAKE, FAKE, 1, 4, 2, 1024, 128, 4, 0, 1, 1, 1, FAKE, 64, None) == B.EWORKSPACE

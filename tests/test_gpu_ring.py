@@ -140,3 +140,88 @@ def test_ring_step_rejects_bad_arguments(cuda_lib):
     with pytest.raises(RingAttnError):  # kv_index out of range
         ring_attention_ring_step(qs[0], ks[0], vs[0], w.S, w.P, 0, 4, True, "striped", w.scale, first=True,
                                  last=True)
+
+
+# ------------------------------------------------------------------ backward ring
+
+def run_backward_ring_sequential(w, q, k, v, out, lse, dout):
+    """Every rank's steps of the backward ring, one after another on one stream: rank r
+    (query shard r) holds KV shard (r + s) mod P at step s; the dK/dV accumulators belong
+    to the KV shard and are handed from rank to rank, the dQ accumulator stays at its rank."""
+    from sequence_exact_attention_ring_b200 import ring_backward_prep, ring_backward_step
+    P = w.P
+    qs, ks, vs, douts = (ring.split_shards(t, P, w.layout) for t in (q, k, v, dout))
+    outs = ring.split_shards(out, P, w.layout)
+    lses = [x.contiguous() for x in ring.split_shards(lse.unsqueeze(-1), P, w.layout)]
+    lses = [x.squeeze(-1).contiguous() for x in lses]
+    wss = [ring_backward_prep(outs[r], lses[r], douts[r], w.S, P, r, w.causal, w.layout) for r in range(P)]
+    f32 = dict(dtype=torch.float32, device="cuda")
+    dq_acc = [torch.full(x.shape, float("nan"), **f32) for x in qs]
+    dk_acc = [torch.full(x.shape, float("nan"), **f32) for x in ks]
+    dv_acc = [torch.full(x.shape, float("nan"), **f32) for x in vs]
+    dq = [torch.empty_like(x) for x in qs]
+    dk = [torch.empty_like(x) for x in ks]
+    dv = [torch.empty_like(x) for x in vs]
+    for s in range(P):
+        for r in range(P):
+            j = (r + s) % P
+            ring_backward_step(qs[r], douts[r], ks[j], vs[j], w.S, P, r, j, wss[r], w.causal, w.layout, w.scale,
+                               parts=3, first=s == 0, last=s == P - 1, dq_acc=dq_acc[r], dk_acc=dk_acc[j],
+                               dv_acc=dv_acc[j], dq=dq[r], dk=dk[j], dv=dv[j])
+    return (ring.join_shards(dq, w.layout), ring.join_shards(dk, w.layout), ring.join_shards(dv, w.layout))
+
+
+BWD_RING_CASES = [
+    # (B, Hq, Hkv, S, P, causal, layout)
+    (1, 2, 2, 1024, 4, True, "striped"),
+    (1, 2, 2, 1024, 4, True, "contiguous"),    # steps with j > i see nothing
+    (2, 4, 2, 768, 3, True, "striped"),        # GQA 2, B = 2
+    (1, 2, 2, 1024, 4, True, "zigzag"),
+    (1, 2, 1, 1000, 4, True, "zigzag"),        # C = 125: not whole tiles
+    (1, 2, 2, 1024, 4, False, "contiguous"),
+    (1, 2, 2, 640, 1, True, "striped"),        # P = 1: first and last in one step
+]
+
+
+@pytest.mark.parametrize("case", BWD_RING_CASES, ids=lambda c: "-".join(map(str, c)))
+def test_backward_ring_steps_match_the_oracle(cuda_lib, case):
+    from test_gpu_backward import assert_grad
+    from sequence_exact_attention_ring_b200 import ring_attention
+    B, Hq, Hkv, S, P, causal, layout = case
+    w = synthetic.custom("bring", "bf16", B, Hq, Hkv, S, 128, P, causal, layout, 331)
+    q, k, v = (t.cuda() for t in synthetic.make_inputs(w, "cpu"))
+    dout = synthetic.make_dout(w, "cpu").cuda()
+    out, lse = ring_attention(q, k, v, P, causal, layout, w.scale)
+    dq, dk, dv = run_backward_ring_sequential(w, q, k, v, out, lse, dout)
+    torch.cuda.synchronize()
+    ref = oracle.attention_backward_reference(q.cpu(), k.cpu(), v.cpu(), dout.cpu(), causal, w.scale)
+    for name, got, r in zip(("dq", "dk", "dv"), (dq, dk, dv), ref):
+        assert_grad(got, r, f"{case} {name}")
+
+
+def test_backward_ring_parts_called_separately_agree(cuda_lib):
+    """Running the dK/dV part and the dQ part as two calls (so the accumulators can leave
+    between them) gives the same bits as one call with both parts."""
+    from sequence_exact_attention_ring_b200 import ring_attention, ring_backward_prep, ring_backward_step
+    w = synthetic.custom("bparts", "bf16", 1, 2, 2, 1024, 128, 4, True, "striped", 337)
+    q, k, v = (t.cuda() for t in synthetic.make_inputs(w, "cpu"))
+    dout = synthetic.make_dout(w, "cpu").cuda()
+    out, lse = ring_attention(q, k, v, w.P, True, "striped", w.scale)
+    qs, ks, vs, douts, outs = (ring.split_shards(t, w.P, "striped") for t in (q, k, v, dout, out))
+    lses = [x.squeeze(-1).contiguous() for x in ring.split_shards(lse.unsqueeze(-1), w.P, "striped")]
+    r, j = 1, 3
+    ws = ring_backward_prep(outs[r], lses[r], douts[r], w.S, w.P, r, True, "striped")
+    res = []
+    for split in (False, True):
+        accs = [torch.zeros(x.shape, dtype=torch.float32, device="cuda") for x in (qs[r], ks[j], vs[j])]
+        kw = dict(first=True, dq_acc=accs[0], dk_acc=accs[1], dv_acc=accs[2])
+        if split:
+            ring_backward_step(qs[r], douts[r], ks[j], vs[j], w.S, w.P, r, j, ws, True, "striped", w.scale, parts=1, **kw)
+            ring_backward_step(qs[r], douts[r], ks[j], vs[j], w.S, w.P, r, j, ws, True, "striped", w.scale, parts=2, **kw)
+        else:
+            ring_backward_step(qs[r], douts[r], ks[j], vs[j], w.S, w.P, r, j, ws, True, "striped", w.scale, parts=3, **kw)
+        torch.cuda.synchronize()
+        res.append([a.clone() for a in accs])
+        assert all(torch.isfinite(a).all() for a in accs)
+    for a, b in zip(*res):
+        assert torch.equal(a, b)

@@ -109,3 +109,65 @@ def test_ring_pass_bookkeeping_with_gloo_ranks(world, direction):
             assert first == (s == 0) and last == (s == world - 1)
             assert own == (s == 0)                            # step 0 uses the rank's own buffers
         assert (k0, v0) == (rank, 100 + rank)                 # the caller's shard is never overwritten
+
+
+def _bwd_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import datetime
+
+    import torch.distributed as dist
+    from sequence_exact_attention_ring_b200 import ring as rg
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        # the rank's KV shard carries its index; each rank adds rank + 1 to dK and 10 (rank + 1) to dV
+        k = torch.full((1, 2, 3, 4), float(rank))
+        v = torch.full((1, 2, 3, 4), float(100 + rank))
+        acc_like = torch.empty((1, 2, 3, 4))
+        seen = []
+
+        def step_kv(s, j, kc, vc, acc_k, acc_v, fin_k, fin_v, first, last):
+            assert float(kc.unique().item()) == j and float(vc.unique().item()) == 100 + j
+            prev_k = 0.0 if first else acc_k.clone()
+            prev_v = 0.0 if first else acc_v.clone()
+            if last:  # finished: tag with the shard index so the test sees where it ends up
+                fin_k.copy_(prev_k + (rank + 1) + 1000 * j)
+                fin_v.copy_(prev_v + 10 * (rank + 1) + 1000 * j)
+            else:
+                acc_k.copy_(prev_k + (rank + 1))
+                acc_v.copy_(prev_v + 10 * (rank + 1))
+            seen.append(("kv", s, j, first, last))
+
+        def step_q(s, j, kc, vc, first, last):
+            seen.append(("q", s, j, first, last))
+
+        dk, dv = rg.run_backward_ring(k, v, acc_like, step_kv, step_q)
+        q.put((rank, seen, float(dk.unique().item()), float(dv.unique().item())))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_backward_ring_accumulators_collect_every_rank_and_return_home(world):
+    """The backward ring (RingAttention deep-architecture article, section "activation
+    checkpointing and memory recomputation"): rank r holds KV shard (r + s) mod world at step s,
+    the dK/dV accumulators travel with it and gather one part from every rank, and the
+    finished gradients of shard r end at rank r."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_bwd_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    total = world * (world + 1) // 2
+    for rank, seen, dk, dv in res:
+        kv = [x for x in seen if x[0] == "kv"]
+        qq = [x for x in seen if x[0] == "q"]
+        assert [x[2] for x in kv] == [(rank + s) % world for s in range(world)]
+        assert [x[2] for x in qq] == [(rank + s) % world for s in range(world)]
+        assert all(x[3] == (x[1] == 0) and x[4] == (x[1] == world - 1) for x in seen)
+        assert dk == total + 1000 * rank and dv == 10 * total + 1000 * rank

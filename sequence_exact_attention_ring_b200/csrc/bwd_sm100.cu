@@ -478,12 +478,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Shared memory of the dQ kernel: a ring of 64-key K or V slots only; Q and dO sit
+// Shared memory of the dQ kernel: a ring of 64-key slots only, each the K step followed
+// by the V step, behind one barrier (one wait per step for the MMA warp); Q and dO sit
 // in tensor memory as the A operands of their products.
 constexpr int kB_OffRing = 0;
-constexpr int kB_SlotsFit = (kSmemLimit - 1024 - 64 - 512 - kB_OffRing) / kStepTileBytes;
-constexpr int kB_Slots = kB_SlotsFit < 12 ? kB_SlotsFit : 12;
-constexpr int kB_OffBar = kB_OffRing + kB_Slots * kStepTileBytes;
+constexpr int kB_SlotBytes = 2 * kStepTileBytes;
+constexpr int kB_SlotsFit = (kSmemLimit - 1024 - 64 - 512 - kB_OffRing) / kB_SlotBytes;
+constexpr int kB_Slots = kB_SlotsFit < 6 ? kB_SlotsFit : 6;
+constexpr int kB_OffBar = kB_OffRing + kB_Slots * kB_SlotBytes;
 constexpr uint32_t kColQ = 384;   // Q tile, bf16 pairs: 64 columns
 constexpr uint32_t kColDO = 448;  // dO tile, bf16 pairs: 64 columns
 // kB_QReady: the eight elementwise warps have written Q and dO into tensor memory
@@ -491,7 +493,7 @@ enum BarB { kB_QReady = 0, kB_SFull = 1, kB_PReady = 3, kB_Done = 5, kB_Drain = 
 constexpr int kB_NumBars = kB_Ring + 2 * kB_Slots;
 constexpr int kB_OffMisc = kB_OffBar + kB_NumBars * 8;
 constexpr int kB_SmemBytes = kB_OffMisc + 64 + 1024;
-static_assert(kB_Slots >= 4, "need two steps of K and V slots");
+static_assert(kB_Slots >= 3, "steps n, n + 1 and n + 2 are held at once");
 static_assert(kB_SmemBytes <= kSmemLimit, "shared memory budget");
 
 // dQ: one CTA per 128-row query tile; keys arrive in steps of 64 along the backward
@@ -555,20 +557,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       int c1, c2;
-      int64_t m = 0;
+      int64_t m = 0;  // steps loaded
       bool ok = true;
       for (TileWalk w = walk_begin_rev(g, U.i, a_hi, TS, anchor, s_lo, s_hi); walk_valid(w) && ok;
-           walk_next(g, w, a_hi, TS)) {
+           walk_next(g, w, a_hi, TS), ++m) {
         tile_coords(g, p.step != 0, w.j, (int64_t)w.kb * TS, c1, c2);
-        for (int kind = 0; kind < 2; ++kind, ++m) {
-          const int slot = slot_of(m);
-          if (!(ok = mbar_wait_backoff<false>(&empty[slot], phase_of(m) ^ 1, wd, kProducerSleepNs))) break;
-          uint8_t* dst = smem + kB_OffRing + slot * kStepTileBytes;
-          mbar_arrive_expect_tx(&full[slot], kStepTileBytes);
-          const CUtensorMap* tm = kind == 0 ? &tm_k : &tm_v;
-          for (int bx = 0; bx < 2; ++bx)
-            tma_load_4d(dst + bx * kStepBoxBytes, tm, &full[slot], bx * BOXW, c1, c2, bh_kv);
-        }
+        const int slot = slot_of(m);
+        if (!(ok = mbar_wait_backoff<false>(&empty[slot], phase_of(m) ^ 1, wd, kProducerSleepNs))) break;
+        uint8_t* dst = smem + kB_OffRing + slot * kB_SlotBytes;
+        mbar_arrive_expect_tx(&full[slot], kB_SlotBytes);
+        for (int bx = 0; bx < 2; ++bx)
+          tma_load_4d(dst + bx * kStepBoxBytes, &tm_k, &full[slot], bx * BOXW, c1, c2, bh_kv);
+        for (int bx = 0; bx < 2; ++bx)
+          tma_load_4d(dst + kStepTileBytes + bx * kStepBoxBytes, &tm_v, &full[slot], bx * BOXW, c1, c2, bh_kv);
       }
       if (!ok) {
         for (int64_t x = (m > kB_Slots ? m - kB_Slots : 0); x < m; ++x)
@@ -580,25 +581,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool issuer = elect_one_sync();
     const uint32_t sbase = smem_u32(smem);
     auto all = [&](bool r) { return __all_sync(0xffffffffu, r); };
-    auto slot_addr = [&](int64_t m) { return sbase + kB_OffRing + slot_of(m) * kStepTileBytes; };
+    auto slot_addr = [&](int64_t n) { return sbase + kB_OffRing + slot_of(n) * kB_SlotBytes; };
     // S = Q K^T and dP = dO V^T of step n into buffer n % 2
     auto issue_sd = [&](int64_t n) -> bool {
-      if (!all(mbar_wait(&full[slot_of(2 * n)], phase_of(2 * n), wd))) return false;
-      if (!all(mbar_wait(&full[slot_of(2 * n + 1)], phase_of(2 * n + 1), wd))) return false;
+      if (!all(mbar_wait(&full[slot_of(n)], phase_of(n), wd))) return false;
       tc_fence_after();
       const int b = (int)(n & 1);
-      const uint64_t bk = smem_desc_sw128(slot_addr(2 * n), 0, 1024);
-      const uint64_t bv = smem_desc_sw128(slot_addr(2 * n + 1), 0, 1024);
+      const uint64_t bk = smem_desc_sw128(slot_addr(n), 0, 1024);
+      const uint64_t bv = smem_desc_sw128(slot_addr(n) + kStepTileBytes, 0, 1024);
 #pragma unroll
       for (int k = 0; k < D / 16; ++k)  // K step k: dims 16k..16k+15 = packed columns 8k..8k+7
         if (issuer) mma_ts(tmem + col_s(b), tmem + kColQ + 8 * k, kmajor64_step(bk, k), kIdescSS64, k > 0);
 #pragma unroll
       for (int k = 0; k < D / 16; ++k)
         if (issuer) mma_ts(tmem + col_dp(b), tmem + kColDO + 8 * k, kmajor64_step(bv, k), kIdescSS64, k > 0);
-      if (issuer) {
-        mma_commit(&bars[kB_SFull + b]);
-        mma_commit(&empty[slot_of(2 * n + 1)]);  // V is no longer needed once dP is done
-      }
+      if (issuer) mma_commit(&bars[kB_SFull + b]);
       return true;
     };
     bool ok = N > 0 && all(mbar_wait(&bars[kB_QReady], 0, wd));
@@ -611,12 +608,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int b = (int)(n & 1);
       if (!(ok = all(mbar_wait(&bars[kB_PReady + b], (uint32_t)((n >> 1) & 1), wd)))) break;
       tc_fence_after();
-      const uint64_t mk = smem_desc_sw128(slot_addr(2 * n), kStepBoxBytes, 1024);
+      const uint64_t mk = smem_desc_sw128(slot_addr(n), kStepBoxBytes, 1024);
 #pragma unroll
       for (int k = 0; k < TS / 16; ++k)  // dQ += dS K
         if (issuer) mma_ts(tmem + kColAcc, tmem + col_s(b) + packed64_step_col(k), mnmajor_step(mk, k), kIdescTS,
                            !(n == 0 && k == 0));
-      if (issuer) mma_commit(&empty[slot_of(2 * n)]);
+      if (issuer) mma_commit(&empty[slot_of(n)]);  // K (dQ) and V (dP) of step n are read
       if (n + 2 < N && !(ok = issue_sd(n + 2))) break;
     }
     if (issuer) {

@@ -258,20 +258,25 @@ __device__ __forceinline__ uint64_t kmajor64_step(uint64_t base, int k) {
 // rows written by the two column halves (32 rows each, 16 packed columns each)
 __device__ __forceinline__ uint32_t packed64_step_col(int k) { return (uint32_t)((k / 2) * 32 + (k % 2) * 8); }
 
-// Shared memory of the dK/dV kernel: K and V tiles, then a ring of query-side slots
-// (a 64-row Q or dO tile followed by its 64 statistics).
+// Shared memory of the dK/dV kernel: K and V tiles, then a ring of query-side slots,
+// each one step's 64-row Q tile, its dO tile and their statistics (lse, Delta) behind
+// one barrier (one wait per step for the MMA warp).
 constexpr int kA_OffK = 0;
 constexpr int kA_OffV = kTileBytes;
 constexpr int kA_OffRing = 2 * kTileBytes;
-constexpr int kA_SlotBytes = ((kStepTileBytes + kStepStatBytes + 1023) / 1024) * 1024;
+constexpr int kA_SlotDO = kStepTileBytes;
+constexpr int kA_SlotLse = 2 * kStepTileBytes;
+constexpr int kA_SlotDelta = kA_SlotLse + kStepStatBytes;
+constexpr int kA_SlotFill = 2 * kStepTileBytes + 2 * kStepStatBytes;
+constexpr int kA_SlotBytes = ((kA_SlotFill + 1023) / 1024) * 1024;
 constexpr int kA_SlotsFit = (kSmemLimit - 1024 - 64 - 512 - kA_OffRing) / kA_SlotBytes;
-constexpr int kA_Slots = kA_SlotsFit < 8 ? kA_SlotsFit : 8;
+constexpr int kA_Slots = kA_SlotsFit < 4 ? kA_SlotsFit : 4;
 constexpr int kA_OffBar = kA_OffRing + kA_Slots * kA_SlotBytes;
 enum BarA { kA_KVFull = 0, kA_STFull = 1, kA_PReady = 3, kA_Done = 5, kA_Drain = 6, kA_Ring = 7 };
 constexpr int kA_NumBars = kA_Ring + 2 * kA_Slots;
 constexpr int kA_OffMisc = kA_OffBar + kA_NumBars * 8;
 constexpr int kA_SmemBytes = kA_OffMisc + 64 + 1024;
-static_assert(kA_Slots >= 4, "need two steps of Q and dO slots");
+static_assert(kA_Slots >= 3, "steps n, n + 1 and n + 2 are held at once");
 static_assert(kA_SmemBytes <= kSmemLimit, "shared memory budget");
 
 // dK/dV: one CTA per 128-key tile; query rows arrive in steps of 64. TMEM holds two
@@ -333,23 +338,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_4d(smem + kA_OffK + bx * kBoxBytes, &tm_k, &bars[kA_KVFull], bx * BOXW, c1, c2, bh_kv);
         tma_load_4d(smem + kA_OffV + bx * kBoxBytes, &tm_v, &bars[kA_KVFull], bx * BOXW, c1, c2, bh_kv);
       }
-      int64_t m = 0;
+      int64_t m = 0;  // steps loaded
       bool ok = true;
-      for (QWalk w = qwalk_begin(g, U, TS, BT, q_only); qwalk_valid(w) && ok; qwalk_next(g, w, TS)) {
+      for (QWalk w = qwalk_begin(g, U, TS, BT, q_only); qwalk_valid(w) && ok; qwalk_next(g, w, TS), ++m) {
         const int bh_q = U.b * g.Hq + U.g * rep + w.hr;
         const int64_t a0 = (int64_t)w.qt * TS;
         tile_coords(g, p.step != 0, w.i, a0, c1, c2);
         const int64_t stat = stat_row(p, bh_q, w.i, a0);
-        for (int kind = 0; kind < 2; ++kind, ++m) {
-          const int slot = slot_of(m);
-          if (!(ok = mbar_wait_backoff<false>(&empty[slot], phase_of(m) ^ 1, wd, kProducerSleepNs))) break;
-          uint8_t* dst = smem + kA_OffRing + slot * kA_SlotBytes;
-          mbar_arrive_expect_tx(&full[slot], kStepTileBytes + kStepStatBytes);
-          const CUtensorMap* tm = kind == 0 ? &tm_q : &tm_do;
-          for (int bx = 0; bx < 2; ++bx)
-            tma_load_4d(dst + bx * kStepBoxBytes, tm, &full[slot], bx * BOXW, c1, c2, bh_q);
-          bulk_load(dst + kStepTileBytes, (kind == 0 ? p.lse2 : p.delta) + stat, kStepStatBytes, &full[slot]);
-        }
+        const int slot = slot_of(m);
+        if (!(ok = mbar_wait_backoff<false>(&empty[slot], phase_of(m) ^ 1, wd, kProducerSleepNs))) break;
+        uint8_t* dst = smem + kA_OffRing + slot * kA_SlotBytes;
+        mbar_arrive_expect_tx(&full[slot], kA_SlotFill);
+        for (int bx = 0; bx < 2; ++bx)
+          tma_load_4d(dst + bx * kStepBoxBytes, &tm_q, &full[slot], bx * BOXW, c1, c2, bh_q);
+        for (int bx = 0; bx < 2; ++bx)
+          tma_load_4d(dst + kA_SlotDO + bx * kStepBoxBytes, &tm_do, &full[slot], bx * BOXW, c1, c2, bh_q);
+        bulk_load(dst + kA_SlotLse, p.lse2 + stat, kStepStatBytes, &full[slot]);
+        bulk_load(dst + kA_SlotDelta, p.delta + stat, kStepStatBytes, &full[slot]);
       }
       if (!ok) {
         // wind down: this CTA's own copies must land before its shared memory goes away
@@ -365,15 +370,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t dK = smem_desc_sw128(sbase + kA_OffK, 0, 1024);
     const uint64_t dV = smem_desc_sw128(sbase + kA_OffV, 0, 1024);
     auto all = [&](bool r) { return __all_sync(0xffffffffu, r); };
-    auto slot_addr = [&](int64_t m) { return sbase + kA_OffRing + slot_of(m) * kA_SlotBytes; };
+    auto slot_addr = [&](int64_t n) { return sbase + kA_OffRing + slot_of(n) * kA_SlotBytes; };
     // S^T = K Q^T and dP^T = V dO^T of step n into buffer n % 2
     auto issue_st = [&](int64_t n) -> bool {
-      if (!all(mbar_wait(&full[slot_of(2 * n)], phase_of(2 * n), wd))) return false;
-      if (!all(mbar_wait(&full[slot_of(2 * n + 1)], phase_of(2 * n + 1), wd))) return false;
+      if (!all(mbar_wait(&full[slot_of(n)], phase_of(n), wd))) return false;
       tc_fence_after();
       const int b = (int)(n & 1);
-      const uint64_t bq = smem_desc_sw128(slot_addr(2 * n), 0, 1024);
-      const uint64_t bd = smem_desc_sw128(slot_addr(2 * n + 1), 0, 1024);
+      const uint64_t bq = smem_desc_sw128(slot_addr(n), 0, 1024);
+      const uint64_t bd = smem_desc_sw128(slot_addr(n) + kA_SlotDO, 0, 1024);
 #pragma unroll
       for (int k = 0; k < D / 16; ++k)
         if (issuer) mma_ss(tmem + col_s(b), kmajor_step(dK, k), kmajor64_step(bq, k), kIdescSS64, k > 0);
@@ -390,8 +394,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int b = (int)(n & 1);
       if (!(ok = all(mbar_wait(&bars[kA_PReady + b], (uint32_t)((n >> 1) & 1), wd)))) break;
       tc_fence_after();
-      const uint64_t mq = smem_desc_sw128(slot_addr(2 * n), kStepBoxBytes, 1024);
-      const uint64_t md = smem_desc_sw128(slot_addr(2 * n + 1), kStepBoxBytes, 1024);
+      const uint64_t mq = smem_desc_sw128(slot_addr(n), kStepBoxBytes, 1024);
+      const uint64_t md = smem_desc_sw128(slot_addr(n) + kA_SlotDO, kStepBoxBytes, 1024);
 #pragma unroll
       for (int k = 0; k < TS / 16; ++k)  // dV += P^T dO
         if (issuer) mma_ts(tmem + kColAcc, tmem + col_s(b) + packed64_step_col(k), mnmajor_step(md, k), kIdescTS,
@@ -400,10 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int k = 0; k < TS / 16; ++k)  // dK += dS^T Q
         if (issuer) mma_ts(tmem + kColAcc + D, tmem + col_dp(b) + packed64_step_col(k), mnmajor_step(mq, k), kIdescTS,
                            !(n == 0 && k == 0));
-      if (issuer) {
-        mma_commit(&empty[slot_of(2 * n)]);
-        mma_commit(&empty[slot_of(2 * n + 1)]);
-      }
+      if (issuer) mma_commit(&empty[slot_of(n)]);
       // buffer b is free for step n + 2 once these products have read its P and dS
       if (n + 2 < N && !(ok = issue_st(n + 2))) break;
     }
@@ -426,13 +427,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     int64_t row0 = 0;  // first row of shard row_i whose token is >= u
     for (QWalk w = qwalk_begin(g, U, TS, BT, q_only); qwalk_valid(w); qwalk_next(g, w, TS), ++n) {
       const int b = (int)(n & 1);
-      const int sq = slot_of(2 * n), sd = slot_of(2 * n + 1);
+      const int sl = slot_of(n);
       if (!(ok = mbar_wait(&bars[kA_STFull + b], (uint32_t)((n >> 1) & 1), wd))) break;
-      // the statistics came with the tiles: wait on their barriers too (already complete)
-      if (!(ok = mbar_wait(&full[sq], phase_of(2 * n), wd) && mbar_wait(&full[sd], phase_of(2 * n + 1), wd))) break;
+      // the statistics came with the tiles: wait on their barrier too (already complete)
+      if (!(ok = mbar_wait(&full[sl], phase_of(n), wd))) break;
       tc_fence_after();
-      const float* lse2c = reinterpret_cast<const float*>(smem + kA_OffRing + sq * kA_SlotBytes + kStepTileBytes);
-      const float* deltac = reinterpret_cast<const float*>(smem + kA_OffRing + sd * kA_SlotBytes + kStepTileBytes);
+      const float* lse2c = reinterpret_cast<const float*>(smem + kA_OffRing + sl * kA_SlotBytes + kA_SlotLse);
+      const float* deltac = reinterpret_cast<const float*>(smem + kA_OffRing + sl * kA_SlotBytes + kA_SlotDelta);
       if (w.i != row_i) {
         row_i = w.i;
         row0 = g.causal ? first_row_at_or_after(g, w.i, u) : 0;

@@ -2,7 +2,7 @@
 """Throughput of exact ring attention on B200: causal-adjusted TFLOP/s, one JSON line.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
-                    [--pass fwd|bwd|decode|merge|ring] [--algo auto|tcgen05|tcgen05_1sm|simt]
+                    [--pass fwd|bwd|decode|merge|ring|ring-bwd] [--algo auto|tcgen05|tcgen05_1sm|simt]
                     [--ring-ranks R]
 
 A step is one ring_attn_fwd call over the whole workload (every query shard folds
@@ -15,7 +15,8 @@ ranks itself.
 
 --pass ring spreads one sequence over ranks instead (the pages' ring: KV shards
 travel between ranks while each rank folds the one it holds): virtual ranks on one
-GPU, or one rank per GPU under torchrun.
+GPU, or one rank per GPU under torchrun. --pass ring-bwd does the same for the
+backward (KV shards and their dK/dV accumulators travel the other way).
 
 --impl reference times the fp64 CPU oracle (the correctness reference) on a
 bounded sample of query rows of the same workload; rank 0 only.
@@ -61,7 +62,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
-    ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd", "decode", "merge", "ring"],
+    ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd", "decode", "merge", "ring", "ring-bwd"],
                     help="fwd: the forward hot path (the headline line); bwd: ring_attn_bwd on the same workload; "
                          "decode: one decode step against the workload's K/V as the cache; ring: the ring spread "
                          "over ranks (virtual ranks on one GPU, or one rank per GPU under torchrun)")
@@ -684,6 +685,112 @@ def run_ring(args, world, rank, local):
     }))
 
 
+RING_BWD_METRIC = "ring spread over ranks (backward): attention backward TFLOP/s (10*D FLOPs per allowed pair)"
+
+
+def run_ring_backward(args, world, rank, local):
+    """The backward ring with the sequence spread over ranks (RingAttention deep-architecture
+    article, section "activation checkpointing and memory recomputation"): every rank keeps
+    its query shard, dO and row statistics; the KV shards travel the other way carrying
+    their dK/dV accumulators; each step is the dK/dV part then the dQ part of
+    ring_attn_bwd_ring_step.
+      one GPU: --ring-ranks virtual ranks (device-to-device copies between their buffers);
+      N GPUs (torchrun): one rank per GPU, NCCL point-to-point.
+    out and lse come from one untimed single-launch forward. Strong scaling: one sequence.
+    Also reports the per-step copy and compute durations and, on one GPU, the single-launch
+    ring_attn_bwd time of the same workload."""
+    from sequence_exact_attention_ring_b200 import binding, ring, ring_attention, ring_attention_backward
+    w = synthetic.get(args.workload)
+    binding.load()
+    dev = torch.device("cuda", local if world > 1 else 0)
+    R = world if world > 1 else args.ring_ranks
+    if w.S % R or (w.layout == "zigzag" and w.S % (2 * R)):
+        raise SystemExit(f"S={w.S} does not split into {R} ring shards")
+    q, k, v = synthetic.make_inputs(w, dev)
+    dout = synthetic.make_dout(w, dev)
+    stream = torch.cuda.current_stream(dev)
+    out, lse = ring_attention(q, k, v, w.P, w.causal, w.layout, w.scale, stream=stream)
+    fused_ms = None
+    if world == 1:
+        ring_attention_backward(q, k, v, out, lse, dout, w.P, w.causal, w.layout, w.scale, stream=stream)
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        ring_attention_backward(q, k, v, out, lse, dout, w.P, w.causal, w.layout, w.scale, stream=stream)
+        f1.record(stream)
+        torch.cuda.synchronize(dev)
+        fused_ms = f0.elapsed_time(f1)
+    shards = [ring.split_shards(t, R, w.layout) for t in (q, k, v, out, dout)]
+    lses = [x.squeeze(-1).contiguous() for x in ring.split_shards(lse.unsqueeze(-1), R, w.layout)]
+    del q, k, v, out, dout, lse
+    qs, ks, vs, outs, douts = shards
+    if world > 1:
+        qs, ks, vs, outs, douts, lses = ([x[rank]] for x in (qs, ks, vs, outs, douts, lses))
+    torch.cuda.synchronize(dev)
+    torch.cuda.empty_cache()
+    if world == 1:
+        vr = ring.VirtualBackwardRing(qs, ks, vs, outs, lses, douts, w.causal, w.layout, w.scale)
+
+        def step(timing=False):
+            return vr.run(timing=timing)
+    else:
+        comm = torch.cuda.Stream(dev)
+
+        def step(timing=False):
+            ring.ring_attention_backward_distributed(qs[0], ks[0], vs[0], outs[0], lses[0], douts[0], w.causal,
+                                                     w.layout, w.scale, stream=stream, comm_stream=comm)
+            return None
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    sampler = ClockSampler(dev.index)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    barrier(world)
+    elapsed = max_over_ranks(t0.elapsed_time(t1), world)
+    overlap = None
+    if world == 1:
+        tm = step(timing=True)
+        torch.cuda.synchronize(dev)
+        comp = [[a.elapsed_time(b) for a, b in per] for per in tm["compute"]]
+        cop = [[a.elapsed_time(b) for a, b in per] for per in tm["copy"]]
+        overlap = {"virtual_ranks": R, "step_ms_wall": elapsed / args.steps,
+                   "fused_single_launch_ms": fused_ms,
+                   "compute_ms_per_rank_max": max(sum(c) for c in comp),
+                   "copy_ms_per_rank_max": max(sum(c) for c in cop) if R > 1 else 0.0,
+                   "copy_ms_per_step_max": max(max(c) for c in cop) if R > 1 else 0.0,
+                   "bytes_per_step_per_rank": (2 * ks[0].numel() * ks[0].element_size()
+                                               + 2 * ks[0].numel() * 4) if R > 1 else 0}
+    flops = 2.5 * w.causal_flops()
+    value = flops * args.steps / (elapsed * 1e-3) / 1e12
+    peaks, peak_src = measured_peaks()
+    peak = float(peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"])
+    clocks_all = gather_objects(clocks, world)
+    if rank != 0:
+        return
+    print(json.dumps({
+        "metric": RING_BWD_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed / args.steps, "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": dict(workload_config(w), **{"pass": "ring-bwd", "ring_ranks": R,
+                                              "transport": "device-to-device copies between virtual ranks"
+                                              if world == 1 else "NCCL point-to-point between GPUs"}),
+        "roofline": {"bound": "tensor", "achieved": value / world, "peak": peak, "unit": "TFLOP/s",
+                     "frac": value / world / peak, "traffic": None,
+                     "peak_source": f"{peak_src} bf16_tflops_sustained",
+                     "kernel": "bwd_prep_kernel, then per ring step bwd_dkdv_kernel and bwd_dq_kernel"},
+        "overlap": overlap,
+        "gpu_launches": (R + 2 * R * R) * args.steps,
+        "clocks": clocks_all[0] if world == 1 else {"per_rank": clocks_all},
+    }))
+
+
 def main():
     args = parse()
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
@@ -700,6 +807,8 @@ def main():
             run_decode(args, world, rank, local)
         elif args.which == "merge":
             run_merge(args, world, rank, local)
+        elif args.which == "ring-bwd":
+            run_ring_backward(args, world, rank, local)
         elif args.which == "ring":
             run_ring(args, world, rank, local)
         else:

@@ -395,3 +395,147 @@ class VirtualRing:
     def results(self):
         """Per-rank (out [B,Hq,Sq,D], lse [B,Hq,Sq]) in shard-local order."""
         return list(zip(self.out, self.lse))
+
+
+class VirtualBackwardRing:
+    """P virtual ranks of the backward ring on one device (the transfers of
+    run_backward_ring as device-to-device copies between the ranks' buffers).
+
+    Rank r keeps query shard r with its dO, out and lse; at step s it holds KV shard
+    j = (r + s) mod P and that shard's dK/dV accumulators (fp32), runs the dK/dV part
+    (ring_attn_bwd_ring_step, parts = KV) then the dQ part (parts = Q) on its compute
+    stream, and its copy stream pulls rank r + 1's K/V (as soon as that rank's step
+    starts reading it) and accumulators (once rank r + 1's dK/dV part is in) into its
+    other buffers. After the last step each rank holds the finished gradients of shard
+    r - 1 and copies them home. Events order the streams; no kernel waits on another.
+    """
+
+    def __init__(self, q_shards, k_shards, v_shards, out_shards, lse_shards, dout_shards, causal=True,
+                 layout="striped", scale=None):
+        self.P = P = len(q_shards)
+        if P < 1 or not all(len(x) == P for x in (k_shards, v_shards, out_shards, lse_shards, dout_shards)):
+            raise ValueError("one shard of each tensor per rank")
+        B, Hq, Sq, D = q_shards[0].shape
+        self.S = P * Sq
+        self.causal, self.layout = causal, layout
+        self.scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+        self.dev = q_shards[0].device
+        self.q, self.k, self.v = list(q_shards), list(k_shards), list(v_shards)
+        self.out, self.lse, self.dout = list(out_shards), list(lse_shards), list(dout_shards)
+        f32 = dict(dtype=torch.float32, device=self.dev)
+        two = 2 if P > 1 else 0
+        self.kv_bufs = [[(torch.empty_like(k_shards[r]), torch.empty_like(v_shards[r])) for _ in range(two)]
+                        for r in range(P)]
+        self.acc_bufs = [[(torch.empty(k_shards[r].shape, **f32), torch.empty(v_shards[r].shape, **f32))
+                          for _ in range(max(two, 1))] for r in range(P)]
+        self.dq_acc = [torch.empty(q_shards[r].shape, **f32) if P > 1 else None for r in range(P)]
+        self.dq = [torch.empty_like(q_shards[r]) for r in range(P)]
+        self.fin = [(torch.empty_like(k_shards[r]), torch.empty_like(v_shards[r])) for r in range(P)]
+        self.dk = [torch.empty_like(k_shards[r]) for r in range(P)]
+        self.dv = [torch.empty_like(v_shards[r]) for r in range(P)]
+        from . import binding as _b
+        wsb = _b.ring_attn_bwd_ring_workspace_bytes(B, Hq, Hq, self.S, D, P, int(causal),
+                                                    {"contiguous": 0, "striped": 1, "zigzag": 2}[layout],
+                                                    _b.DTYPE_BF16)
+        if wsb == 0:
+            raise _b.RingAttnError(_b.EINVAL, "ring_attn_bwd_ring_workspace_bytes")
+        self.ws = [torch.zeros(wsb, dtype=torch.uint8, device=self.dev) for _ in range(P)]
+        self.compute = [torch.cuda.Stream(self.dev) for _ in range(P)]
+        self.copy = [torch.cuda.Stream(self.dev) for _ in range(P)]
+
+    def _kv(self, r, s):
+        return (self.k[r], self.v[r]) if s == 0 else self.kv_bufs[r][(s - 1) % 2]
+
+    def _acc(self, r, s):
+        return self.acc_bufs[r][s % 2] if self.P > 1 else self.acc_bufs[r][0]
+
+    def run(self, timing: bool = False):
+        """Issue the prep and every step of every rank; the caller's current stream waits
+        for all of it. With timing, returns per-step (start, end) CUDA events {"compute":
+        per rank, "copy": per rank, two per step: K/V, then the accumulators}; else None."""
+        from .api import ring_backward_prep, ring_backward_step
+
+        P = self.P
+        caller = torch.cuda.current_stream(self.dev)
+        for st in self.compute + self.copy:
+            st.wait_stream(caller)
+        kv_done = [[None] * P for _ in range(P)]     # dK/dV part of (rank, step) done
+        comp_done = [[None] * P for _ in range(P)]   # both parts done
+        copy_kv = [[None] * P for _ in range(P)]
+        copy_acc = [[None] * P for _ in range(P)]
+        tm = {"compute": [[] for _ in range(P)], "copy": [[] for _ in range(P)]} if timing else None
+
+        def ev(stream):
+            e = torch.cuda.Event(enable_timing=timing)
+            e.record(stream)
+            return e
+
+        for r in range(P):
+            ring_backward_prep(self.out[r], self.lse[r], self.dout[r], self.S, P, r, self.causal, self.layout,
+                               workspace=self.ws[r], stream=self.compute[r])
+        for s in range(P):
+            first, last = s == 0, s == P - 1
+            for r in range(P):
+                cs = self.compute[r]
+                if s > 0:
+                    cs.wait_event(copy_kv[r][s - 1])
+                    cs.wait_event(copy_acc[r][s - 1])
+                j = (r + s) % P
+                kc, vc = self._kv(r, s)
+                ak, av = self._acc(r, s)
+                fk, fv = self.fin[r]
+                t0 = ev(cs) if timing else None
+                ring_backward_step(self.q[r], self.dout[r], kc, vc, self.S, P, r, j, self.ws[r], self.causal,
+                                   self.layout, self.scale, parts=1, first=first, last=last, dk_acc=ak, dv_acc=av,
+                                   dk=fk, dv=fv, stream=cs)
+                kv_done[r][s] = ev(cs)
+                ring_backward_step(self.q[r], self.dout[r], kc, vc, self.S, P, r, j, self.ws[r], self.causal,
+                                   self.layout, self.scale, parts=2, first=first, last=last,
+                                   dq_acc=self.dq_acc[r], dq=self.dq[r], stream=cs)
+                comp_done[r][s] = ev(cs)
+                if timing:
+                    tm["compute"][r].append((t0, comp_done[r][s]))
+            if last:
+                break
+            for r in range(P):
+                src, dst_of = (r + 1) % P, (r - 1) % P  # blocks move to rank - 1
+                xs = self.copy[r]
+                if s > 0:
+                    xs.wait_event(comp_done[r][s - 1])    # this rank read the buffers at step s - 1
+                    xs.wait_event(copy_kv[dst_of][s - 1])  # rank r - 1 copied them out at step s - 1
+                    xs.wait_event(copy_acc[dst_of][s - 1])
+                    xs.wait_event(copy_kv[src][s - 1])     # the source K/V were filled at step s - 1
+                t0 = ev(xs) if timing else None
+                nk, nv = self.kv_bufs[r][s % 2]
+                sk, sv = self._kv(src, s)
+                with torch.cuda.stream(xs):
+                    nk.copy_(sk, non_blocking=True)
+                    nv.copy_(sv, non_blocking=True)
+                copy_kv[r][s] = ev(xs)
+                if timing:
+                    tm["copy"][r].append((t0, copy_kv[r][s]))
+                xs.wait_event(kv_done[src][s])  # the accumulators leave once their part is in
+                t0 = ev(xs) if timing else None
+                na, nb = self._acc(r, s + 1)
+                sa, sb = self._acc(src, s)
+                with torch.cuda.stream(xs):
+                    na.copy_(sa, non_blocking=True)
+                    nb.copy_(sb, non_blocking=True)
+                copy_acc[r][s] = ev(xs)
+                if timing:
+                    tm["copy"][r].append((t0, copy_acc[r][s]))
+        # home: rank r finished shard r - 1 (r itself when P = 1); rank r pulls its own from rank r + 1
+        for r in range(P):
+            src = (r + 1) % P
+            xs = self.copy[r]
+            xs.wait_event(comp_done[src][P - 1])
+            with torch.cuda.stream(xs):
+                self.dk[r].copy_(self.fin[src][0], non_blocking=True)
+                self.dv[r].copy_(self.fin[src][1], non_blocking=True)
+        for st in self.compute + self.copy:
+            caller.wait_stream(st)
+        return tm
+
+    def results(self):
+        """Per-rank (dq [B,Hq,Sq,D], dk [B,Hkv,Sq,D], dv [B,Hkv,Sq,D]) in shard-local order."""
+        return list(zip(self.dq, self.dk, self.dv))

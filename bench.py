@@ -791,6 +791,24 @@ def run_ring_backward(args, world, rank, local):
     }))
 
 
+def dispatch(args, world, rank, local):
+    """Runs the arm and pass the arguments select."""
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+    elif args.which == "bwd":
+        run_backward(args, world, rank, local)
+    elif args.which == "decode":
+        run_decode(args, world, rank, local)
+    elif args.which == "merge":
+        run_merge(args, world, rank, local)
+    elif args.which == "ring-bwd":
+        run_ring_backward(args, world, rank, local)
+    elif args.which == "ring":
+        run_ring(args, world, rank, local)
+    else:
+        run_ours(args, world, rank, local)
+
+
 def main():
     args = parse()
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
@@ -799,20 +817,7 @@ def main():
     if world != args.gpus:
         raise SystemExit(f"--gpus {args.gpus} but {world} ranks were launched")
     try:
-        if args.impl == "reference":
-            run_reference(args, world, rank)
-        elif args.which == "bwd":
-            run_backward(args, world, rank, local)
-        elif args.which == "decode":
-            run_decode(args, world, rank, local)
-        elif args.which == "merge":
-            run_merge(args, world, rank, local)
-        elif args.which == "ring-bwd":
-            run_ring_backward(args, world, rank, local)
-        elif args.which == "ring":
-            run_ring(args, world, rank, local)
-        else:
-            run_ours(args, world, rank, local)
+        dispatch(args, world, rank, local)
     finally:
         if world > 1:
             import torch.distributed as dist

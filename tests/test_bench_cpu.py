@@ -135,3 +135,20 @@ def test_rank_count_must_match_the_gpus_flag():
                         "--workload", "c1_fp32_s1k", "--steps", "1", "--warmup", "0"],
                        capture_output=True, text=True, timeout=300, cwd=ROOT, env=env)
     assert r.returncode != 0 and "2 but 1 ranks" in (r.stderr + r.stdout)
+
+
+def test_every_pass_is_accepted_and_dispatched(monkeypatch):
+    """Each --pass value parses and reaches its own runner (the runners themselves need a GPU)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    called = []
+    for name in ("run_ours", "run_backward", "run_decode", "run_merge", "run_ring", "run_ring_backward"):
+        monkeypatch.setattr(bench, name, lambda *a, _n=name, **k: called.append(_n))
+    for which, runner in (("fwd", "run_ours"), ("bwd", "run_backward"), ("decode", "run_decode"),
+                          ("merge", "run_merge"), ("ring", "run_ring"), ("ring-bwd", "run_ring_backward")):
+        monkeypatch.setattr(sys, "argv", ["bench.py", "--pass", which, "--ring-ranks", "4"])
+        args = bench.parse()
+        assert args.which == which and args.ring_ranks == 4
+        called.clear()
+        bench.dispatch(args, 1, 0, 0)
+        assert called == [runner]

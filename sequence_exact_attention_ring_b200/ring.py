@@ -33,6 +33,7 @@ from __future__ import annotations
 
 import contextlib
 import math
+from typing import NamedTuple
 
 import torch
 
@@ -297,16 +298,118 @@ def ring_attention_backward_distributed(q_shard, k_shard, v_shard, out_shard, ls
 
 # ------------------------------------------------------------------ virtual ranks on one device
 
+class PlanOp(NamedTuple):
+    """One operation of a virtual ring, in issue order.
+
+    name:   (kind, rank, step) (step -1 for the per-rank operations before and after the
+            steps); unique within a plan.
+    stream: ("compute", rank) or ("copy", rank). Operations of one stream run in order.
+    reads, writes: the buffers it touches (names as in the plan builders).
+    waits:  names of earlier operations whose completion it waits for (an event recorded
+            right after each one was issued)."""
+    name: tuple
+    stream: tuple
+    reads: tuple
+    writes: tuple
+    waits: tuple
+
+
+def forward_ring_plan(P: int) -> list:
+    """The operations of VirtualRing.run: P virtual ranks of the forward ring.
+
+    Buffers: ("kv", r) is rank r's own K/V shard, ("buf", r, i) its two receive buffers,
+    ("state", r) its running state and output. Step s of rank r ("step") folds the shard
+    it holds, (r - s) mod P (RingAttention deep-architecture article, section 2); its copy
+    ("copy") pulls rank r - 1's current shard into buffer s % 2, which rank r holds at
+    step s + 1. A copy waits for this rank's step s - 1 (which read the buffer), for rank
+    r + 1's copy at s - 1 (which read it too) and for rank r - 1's copy at s - 1 (which
+    filled the source); a step waits for the copy that filled what it reads."""
+    def cur(r, s):
+        return ("kv", r) if s == 0 else ("buf", r, (s - 1) % 2)
+
+    ops = []
+    for s in range(P):
+        for r in range(P):
+            waits = (("copy", r, s - 1),) if s > 0 else ()
+            reads = (cur(r, s),) if s == 0 else (cur(r, s), ("state", r))
+            ops.append(PlanOp(("step", r, s), ("compute", r), reads, (("state", r),), waits))
+        if s + 1 < P:
+            for r in range(P):
+                prev, nxt = (r - 1) % P, (r + 1) % P
+                waits = (("step", r, s - 1), ("copy", nxt, s - 1), ("copy", prev, s - 1)) if s > 0 else ()
+                ops.append(PlanOp(("copy", r, s), ("copy", r), (cur(prev, s),), (("buf", r, s % 2),), waits))
+    return ops
+
+
+def backward_ring_plan(P: int) -> list:
+    """The operations of VirtualBackwardRing.run: P virtual ranks of the backward ring.
+
+    Buffers: ("in", r) rank r's query-side inputs (q, dO, out, lse), ("stats", r) its row
+    statistics, ("kv", r) its own K/V shard, ("kvbuf", r, i) two receive buffers,
+    ("acc", r, i) two dK/dV accumulator buffers (one when P = 1), ("dq", r) its dQ
+    accumulator and output, ("fin", r) the finished dK/dV of the shard it ends with,
+    ("home", r) its own dK/dV. At step s rank r holds KV shard (r + s) mod P (the backward
+    ring of the RingAttention deep-architecture article, section "activation checkpointing
+    and memory recomputation") with its accumulators: "step_kv" folds rank r's query shard
+    into them (on the last step into "fin"), "step_q" folds the shard into rank r's dQ.
+    Rank r's copies pull rank r + 1's K/V ("copy_kv") and, once rank r + 1's step_kv is
+    in, its accumulators ("copy_acc"); "home" pulls rank r's finished gradients from rank
+    r + 1 after the last step."""
+    def kv(r, s):
+        return ("kv", r) if s == 0 else ("kvbuf", r, (s - 1) % 2)
+
+    def acc(r, s):
+        return ("acc", r, s % 2) if P > 1 else ("acc", r, 0)
+
+    ops = [PlanOp(("prep", r, -1), ("compute", r), (("in", r),), (("stats", r),), ()) for r in range(P)]
+    for s in range(P):
+        first, last = s == 0, s == P - 1
+        for r in range(P):
+            waits = (("copy_kv", r, s - 1), ("copy_acc", r, s - 1)) if s > 0 else ()
+            reads = (("in", r), ("stats", r), kv(r, s)) + (() if first else (acc(r, s),))
+            ops.append(PlanOp(("step_kv", r, s), ("compute", r), reads, (("fin", r),) if last else (acc(r, s),),
+                              waits))
+            reads = (("in", r), ("stats", r), kv(r, s)) + (() if first else (("dq", r),))
+            ops.append(PlanOp(("step_q", r, s), ("compute", r), reads, (("dq", r),), ()))
+        if last:
+            break
+        for r in range(P):
+            src, dst = (r + 1) % P, (r - 1) % P  # blocks move to rank - 1
+            waits = (("step_q", r, s - 1), ("copy_kv", dst, s - 1), ("copy_acc", dst, s - 1),
+                     ("copy_kv", src, s - 1)) if s > 0 else ()
+            ops.append(PlanOp(("copy_kv", r, s), ("copy", r), (kv(src, s),), (("kvbuf", r, s % 2),), waits))
+            ops.append(PlanOp(("copy_acc", r, s), ("copy", r), (acc(src, s),), (acc(r, s + 1),),
+                              (("step_kv", src, s),)))
+    for r in range(P):
+        src = (r + 1) % P
+        ops.append(PlanOp(("home", r, -1), ("copy", r), (("fin", src),), (("home", r),), (("step_q", src, P - 1),)))
+    return ops
+
+
+def _issue_plan(ops, streams, execute, timing: bool):
+    """Issues `ops` in order: each waits for the events of its `waits`, runs execute(op)
+    on its stream, then records its event. Returns {name: event}."""
+    events = {}
+    for op in ops:
+        stream = streams[op.stream]
+        for w in op.waits:
+            stream.wait_event(events[w])
+        with torch.cuda.stream(stream):
+            execute(op, stream)
+        e = torch.cuda.Event(enable_timing=timing)
+        e.record(stream)
+        events[op.name] = e
+    return events
+
+
 class VirtualRing:
     """P virtual ranks of the forward ring on one device, each with its own query shard,
     KV double buffer, running state, workspace, compute stream and copy stream.
 
-    run() issues the P steps of every rank. Rank r's step s folds the KV shard it holds
-    into its state on its compute stream; meanwhile its copy stream pulls the previous
-    rank's current shard into its other buffer (a device-to-device copy). Events order
-    the streams: a copy into a buffer waits for the step and for the neighbour's copy
-    that read it; a step waits for the copy that filled its buffer; a copy waits for the
-    copy that filled its source. No kernel waits on another kernel.
+    run() issues forward_ring_plan(P): rank r's step s folds the KV shard it holds into
+    its state on its compute stream; meanwhile its copy stream pulls the previous rank's
+    current shard into its other buffer (a device-to-device copy). Events order the
+    streams as the plan says; no kernel waits on another kernel.
     """
 
     def __init__(self, q_shards, k_shards, v_shards, causal=True, layout="striped", scale=None):
@@ -336,6 +439,7 @@ class VirtualRing:
         self.ws = [torch.zeros(wsb, dtype=torch.uint8, device=self.dev) for _ in range(P)]
         self.compute = [torch.cuda.Stream(self.dev) for _ in range(P)]
         self.copy = [torch.cuda.Stream(self.dev) for _ in range(P)]
+        self.plan = forward_ring_plan(P)
 
     def _cur(self, r, s):
         return (self.k[r], self.v[r]) if s == 0 else self.bufs[r][(s - 1) % 2]
@@ -347,49 +451,36 @@ class VirtualRing:
         per rank, "copy": likewise} for the overlap measurement; else None."""
         P = self.P
         caller = torch.cuda.current_stream(self.dev)
-        for st in self.compute + self.copy:
+        streams = {("compute", r): self.compute[r] for r in range(P)}
+        streams.update({("copy", r): self.copy[r] for r in range(P)})
+        for st in streams.values():
             st.wait_stream(caller)
-        comp_done = [[None] * P for _ in range(P)]
-        copy_done = [[None] * P for _ in range(P)]
         tm = {"compute": [[] for _ in range(P)], "copy": [[] for _ in range(P)]} if timing else None
+        starts = {}
 
-        def ev(stream):
-            e = torch.cuda.Event(enable_timing=timing)
-            e.record(stream)
-            return e
-
-        for s in range(P):
-            for r in range(P):
-                cs = self.compute[r]
-                if s > 0:
-                    cs.wait_event(copy_done[r][s - 1])
+        def execute(op, stream):
+            kind, r, s = op.name
+            if timing:
+                starts[op.name] = torch.cuda.Event(enable_timing=True)
+                starts[op.name].record(stream)
+            if kind == "step":
                 kc, vc = self._cur(r, s)
-                t0 = ev(cs) if timing else None
                 ring_attention_ring_step(self.q[r], kc, vc, self.S, P, r, (r - s) % P, self.causal, self.layout,
-                                         self.scale, s == 0, s == P - 1, self.o_acc[r], self.lse_acc[r], self.out[r],
-                                         self.lse[r], workspace=self.ws[r], stream=cs)
-                comp_done[r][s] = ev(cs)
-                if timing:
-                    tm["compute"][r].append((t0, comp_done[r][s]))
-            if s + 1 < P:
-                for r in range(P):
-                    prev, nxt_rank = (r - 1) % P, (r + 1) % P
-                    xs = self.copy[r]
-                    if s > 0:
-                        xs.wait_event(comp_done[r][s - 1])         # this buffer was read by step s - 1
-                        xs.wait_event(copy_done[prev][s - 1])      # the source was filled at step s - 1
-                        xs.wait_event(copy_done[nxt_rank][s - 1])  # the next rank read this buffer at s - 1
-                    src_k, src_v = self._cur(prev, s)
-                    dst_k, dst_v = self.bufs[r][s % 2]
-                    t0 = ev(xs) if timing else None
-                    with torch.cuda.stream(xs):
-                        dst_k.copy_(src_k, non_blocking=True)
-                        dst_v.copy_(src_v, non_blocking=True)
-                    copy_done[r][s] = ev(xs)
-                    if timing:
-                        tm["copy"][r].append((t0, copy_done[r][s]))
-        for st in self.compute + self.copy:
+                                         self.scale, s == 0, s == P - 1, self.o_acc[r], self.lse_acc[r],
+                                         self.out[r], self.lse[r], workspace=self.ws[r], stream=stream)
+            else:
+                src_k, src_v = self._cur((r - 1) % P, s)
+                dst_k, dst_v = self.bufs[r][s % 2]
+                dst_k.copy_(src_k, non_blocking=True)
+                dst_v.copy_(src_v, non_blocking=True)
+
+        events = _issue_plan(self.plan, streams, execute, timing)
+        for st in streams.values():
             caller.wait_stream(st)
+        if timing:
+            for op in self.plan:
+                kind, r, _ = op.name
+                tm["compute" if kind == "step" else "copy"][r].append((starts[op.name], events[op.name]))
         return tm
 
     def results(self):
@@ -401,13 +492,13 @@ class VirtualBackwardRing:
     """P virtual ranks of the backward ring on one device (the transfers of
     run_backward_ring as device-to-device copies between the ranks' buffers).
 
-    Rank r keeps query shard r with its dO, out and lse; at step s it holds KV shard
-    j = (r + s) mod P and that shard's dK/dV accumulators (fp32), runs the dK/dV part
-    (ring_attn_bwd_ring_step, parts = KV) then the dQ part (parts = Q) on its compute
-    stream, and its copy stream pulls rank r + 1's K/V (as soon as that rank's step
-    starts reading it) and accumulators (once rank r + 1's dK/dV part is in) into its
-    other buffers. After the last step each rank holds the finished gradients of shard
-    r - 1 and copies them home. Events order the streams; no kernel waits on another.
+    run() issues backward_ring_plan(P). Rank r keeps query shard r with its dO, out and
+    lse; at step s it holds KV shard j = (r + s) mod P and that shard's dK/dV
+    accumulators (fp32), runs the dK/dV part (ring_attn_bwd_ring_step, parts = KV) then
+    the dQ part (parts = Q) on its compute stream, and its copy stream pulls rank r + 1's
+    K/V and (once rank r + 1's dK/dV part is in) accumulators into its other buffers.
+    After the last step each rank holds the finished gradients of shard r - 1 and copies
+    them home. Events order the streams; no kernel waits on another.
     """
 
     def __init__(self, q_shards, k_shards, v_shards, out_shards, lse_shards, dout_shards, causal=True,
@@ -442,6 +533,7 @@ class VirtualBackwardRing:
         self.ws = [torch.zeros(wsb, dtype=torch.uint8, device=self.dev) for _ in range(P)]
         self.compute = [torch.cuda.Stream(self.dev) for _ in range(P)]
         self.copy = [torch.cuda.Stream(self.dev) for _ in range(P)]
+        self.plan = backward_ring_plan(P)
 
     def _kv(self, r, s):
         return (self.k[r], self.v[r]) if s == 0 else self.kv_bufs[r][(s - 1) % 2]
@@ -450,90 +542,66 @@ class VirtualBackwardRing:
         return self.acc_bufs[r][s % 2] if self.P > 1 else self.acc_bufs[r][0]
 
     def run(self, timing: bool = False):
-        """Issue the prep and every step of every rank; the caller's current stream waits
-        for all of it. With timing, returns per-step (start, end) CUDA events {"compute":
-        per rank, "copy": per rank, two per step: K/V, then the accumulators}; else None."""
+        """Issue the plan; the caller's current stream waits for all of it. With timing,
+        returns (start, end) CUDA events {"compute": per rank, one per step (both parts),
+        "copy": per rank, two per step (K/V, then the accumulators)}; else None."""
         from .api import ring_backward_prep, ring_backward_step
 
         P = self.P
         caller = torch.cuda.current_stream(self.dev)
-        for st in self.compute + self.copy:
+        streams = {("compute", r): self.compute[r] for r in range(P)}
+        streams.update({("copy", r): self.copy[r] for r in range(P)})
+        for st in streams.values():
             st.wait_stream(caller)
-        kv_done = [[None] * P for _ in range(P)]     # dK/dV part of (rank, step) done
-        comp_done = [[None] * P for _ in range(P)]   # both parts done
-        copy_kv = [[None] * P for _ in range(P)]
-        copy_acc = [[None] * P for _ in range(P)]
         tm = {"compute": [[] for _ in range(P)], "copy": [[] for _ in range(P)]} if timing else None
+        starts = {}
 
-        def ev(stream):
-            e = torch.cuda.Event(enable_timing=timing)
-            e.record(stream)
-            return e
-
-        for r in range(P):
-            ring_backward_prep(self.out[r], self.lse[r], self.dout[r], self.S, P, r, self.causal, self.layout,
-                               workspace=self.ws[r], stream=self.compute[r])
-        for s in range(P):
+        def execute(op, stream):
+            kind, r, s = op.name
+            if timing:
+                starts[op.name] = torch.cuda.Event(enable_timing=True)
+                starts[op.name].record(stream)
             first, last = s == 0, s == P - 1
-            for r in range(P):
-                cs = self.compute[r]
-                if s > 0:
-                    cs.wait_event(copy_kv[r][s - 1])
-                    cs.wait_event(copy_acc[r][s - 1])
-                j = (r + s) % P
+            if kind == "prep":
+                ring_backward_prep(self.out[r], self.lse[r], self.dout[r], self.S, P, r, self.causal, self.layout,
+                                   workspace=self.ws[r], stream=stream)
+            elif kind == "step_kv":
                 kc, vc = self._kv(r, s)
                 ak, av = self._acc(r, s)
                 fk, fv = self.fin[r]
-                t0 = ev(cs) if timing else None
-                ring_backward_step(self.q[r], self.dout[r], kc, vc, self.S, P, r, j, self.ws[r], self.causal,
-                                   self.layout, self.scale, parts=1, first=first, last=last, dk_acc=ak, dv_acc=av,
-                                   dk=fk, dv=fv, stream=cs)
-                kv_done[r][s] = ev(cs)
-                ring_backward_step(self.q[r], self.dout[r], kc, vc, self.S, P, r, j, self.ws[r], self.causal,
-                                   self.layout, self.scale, parts=2, first=first, last=last,
-                                   dq_acc=self.dq_acc[r], dq=self.dq[r], stream=cs)
-                comp_done[r][s] = ev(cs)
-                if timing:
-                    tm["compute"][r].append((t0, comp_done[r][s]))
-            if last:
-                break
-            for r in range(P):
-                src, dst_of = (r + 1) % P, (r - 1) % P  # blocks move to rank - 1
-                xs = self.copy[r]
-                if s > 0:
-                    xs.wait_event(comp_done[r][s - 1])    # this rank read the buffers at step s - 1
-                    xs.wait_event(copy_kv[dst_of][s - 1])  # rank r - 1 copied them out at step s - 1
-                    xs.wait_event(copy_acc[dst_of][s - 1])
-                    xs.wait_event(copy_kv[src][s - 1])     # the source K/V were filled at step s - 1
-                t0 = ev(xs) if timing else None
-                nk, nv = self.kv_bufs[r][s % 2]
-                sk, sv = self._kv(src, s)
-                with torch.cuda.stream(xs):
-                    nk.copy_(sk, non_blocking=True)
-                    nv.copy_(sv, non_blocking=True)
-                copy_kv[r][s] = ev(xs)
-                if timing:
-                    tm["copy"][r].append((t0, copy_kv[r][s]))
-                xs.wait_event(kv_done[src][s])  # the accumulators leave once their part is in
-                t0 = ev(xs) if timing else None
+                ring_backward_step(self.q[r], self.dout[r], kc, vc, self.S, P, r, (r + s) % P, self.ws[r],
+                                   self.causal, self.layout, self.scale, parts=1, first=first, last=last,
+                                   dk_acc=ak, dv_acc=av, dk=fk, dv=fv, stream=stream)
+            elif kind == "step_q":
+                kc, vc = self._kv(r, s)
+                ring_backward_step(self.q[r], self.dout[r], kc, vc, self.S, P, r, (r + s) % P, self.ws[r],
+                                   self.causal, self.layout, self.scale, parts=2, first=first, last=last,
+                                   dq_acc=self.dq_acc[r], dq=self.dq[r], stream=stream)
+            elif kind == "copy_kv":
+                dk_, dv_ = self.kv_bufs[r][s % 2]
+                sk, sv = self._kv((r + 1) % P, s)
+                dk_.copy_(sk, non_blocking=True)
+                dv_.copy_(sv, non_blocking=True)
+            elif kind == "copy_acc":
                 na, nb = self._acc(r, s + 1)
-                sa, sb = self._acc(src, s)
-                with torch.cuda.stream(xs):
-                    na.copy_(sa, non_blocking=True)
-                    nb.copy_(sb, non_blocking=True)
-                copy_acc[r][s] = ev(xs)
-                if timing:
-                    tm["copy"][r].append((t0, copy_acc[r][s]))
-        # home: rank r finished shard r - 1 (r itself when P = 1); rank r pulls its own from rank r + 1
-        for r in range(P):
-            src = (r + 1) % P
-            xs = self.copy[r]
-            xs.wait_event(comp_done[src][P - 1])
-            with torch.cuda.stream(xs):
+                sa, sb = self._acc((r + 1) % P, s)
+                na.copy_(sa, non_blocking=True)
+                nb.copy_(sb, non_blocking=True)
+            else:  # home
+                src = (r + 1) % P
                 self.dk[r].copy_(self.fin[src][0], non_blocking=True)
                 self.dv[r].copy_(self.fin[src][1], non_blocking=True)
-        for st in self.compute + self.copy:
+
+        events = _issue_plan(self.plan, streams, execute, timing)
+        for st in streams.values():
             caller.wait_stream(st)
+        if timing:
+            for op in self.plan:
+                kind, r, s = op.name
+                if kind == "step_q":
+                    tm["compute"][r].append((starts[("step_kv", r, s)], events[op.name]))
+                elif kind in ("copy_kv", "copy_acc"):
+                    tm["copy"][r].append((starts[op.name], events[op.name]))
         return tm
 
     def results(self):

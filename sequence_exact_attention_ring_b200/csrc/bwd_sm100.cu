@@ -29,6 +29,10 @@
 // Both keep two TMEM buffers of the 64-column score and dP tiles, so the tensor cores
 // compute step n + 1 (and finish step n - 1's accumulation) while the elementwise
 // warps work on step n.
+// The streamed operands of a step (dK/dV: the Q and dO steps and their statistics; dQ:
+// the K and V steps) share one shared-memory ring slot behind one barrier: every
+// barrier wait costs the MMA warp on the order of a hundred clocks, during which the
+// tensor pipe, which queues only a few instructions, drains.
 // Splitting dQ from dK/dV recomputes S and dP once more (7 instead of 5 GEMMs) and
 // in exchange needs no atomic accumulation anywhere.
 //
